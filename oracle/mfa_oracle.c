@@ -1,0 +1,228 @@
+/*
+ * mfa_oracle.c -- plain, slow, float64 CPU oracle for MFA decode attention and
+ * the MFA low-rank query projection.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
+ * this file: only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg use it. It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (Step-3 page, "Key points -> Architecture"): every decode
+ * token has 64 query heads of dimension 256 that all attend over ONE shared key
+ * head and ONE shared value head of dimension 256; the queries come out of a
+ * 2048-wide low-rank bottleneck fed by the 7168-wide hidden state. The pages
+ * print no attention formula; the plain reading used here is scaled dot-product
+ * attention with a softmax over the cached tokens:
+ *
+ *     s[t]      = scale * sum_i q[b,h,i] * K_b[t,i]           (t < L_b)
+ *     w[t]      = exp(s[t] - max_u s[u]) / sum_u exp(s[u] - max_u s[u])
+ *     out[b,h,:] = sum_t w[t] * V_b[t,:]
+ *     lse[b,h]   = max_u s[u] + log(sum_u exp(s[u] - max_u s[u]))
+ *
+ * K_b / V_b are either a contiguous per-sequence slab or are gathered through a
+ * page table (PagedAttention, cited in the Step-3 page's reference list): token
+ * t of sequence b lives in physical page page_table[b][t / page_size], row
+ * t % page_size. FP8 caches hold E4M3 codes (the pages deploy attention in FP8);
+ * the dequantised value is decode_e4m3(code) * k_scale (resp. v_scale).
+ * An empty sequence (L_b = 0) has no softmax; this oracle defines its output as
+ * zeros and its lse as -inf.
+ *
+ * The projection (same page, "Queries pass through a 2048-dim low-rank
+ * bottleneck") is q = (x * W_qa) * W_qb with no bias, norm or activation, all in
+ * float64 from the bf16 inputs.
+ *
+ * Every input arrives as the exact bit pattern the GPU sees (bf16 bits or E4M3
+ * codes) and is up-converted exactly to double here; all arithmetic is double.
+ *
+ * Build: gcc -O2 -fno-fast-math -fopenmp -shared -fPIC mfa_oracle.c -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_BF16 = 0, OR_F32 = 1, OR_E4M3 = 2 };
+
+/* bf16 is the top half of an IEEE binary32: shift into place, reinterpret. */
+static double bf16_bits_to_double(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* OCP FP8 E4M3 ("e4m3fn"): 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+ * bits, no infinities; S.1111.111 is NaN. Exponent field 0 is subnormal:
+ * 2^-6 * m/8. Otherwise 2^(e-7) * (1 + m/8). */
+double mfa_oracle_e4m3_to_double(uint8_t code) {
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double mag;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* One cached element as a double (before any per-tensor scale). */
+static double cache_elem(const void* base, int dtype, int64_t idx) {
+    if (dtype == OR_E4M3) return mfa_oracle_e4m3_to_double(((const uint8_t*)base)[idx]);
+    if (dtype == OR_F32) return (double)((const float*)base)[idx];
+    return bf16_bits_to_double(((const uint16_t*)base)[idx]);
+}
+
+/* Element index of K_b[t][i] (same for V): contiguous [B][Lmax][D] addressed by
+ * strides, or paged [num_pages][page_size][D] through the page table. Returns -1
+ * on an out-of-range page id. */
+static int64_t cache_index(int b, int t, int i, int D, int64_t batch_stride, int64_t token_stride,
+                           const int32_t* page_table, int max_pages, int page_size, int num_pages) {
+    if (!page_table) return (int64_t)b * batch_stride + (int64_t)t * token_stride + i;
+    int logical_page = t / page_size;
+    int32_t phys = page_table[(int64_t)b * max_pages + logical_page];
+    if (phys < 0 || phys >= num_pages) return -1;
+    return ((int64_t)phys * page_size + (t % page_size)) * D + i;
+}
+
+/*
+ * Decode attention for the (b, h) pairs listed in sel_b/sel_h (nsel of them), or
+ * for all B*H pairs when sel_b == NULL (then out is [B][H][D], lse is [B][H]).
+ * With a selection, out is [nsel][D] and lse is [nsel].
+ *
+ * q: [B][H][D] bf16 bits. k, v: cache of kv_dtype (0 bf16, 1 f32, 2 e4m3).
+ * Contiguous caches (page_table == NULL) are addressed as b*batch_stride +
+ * t*token_stride + i (element units). seq_lens[b] tokens of sequence b are used.
+ * Returns 0, or -1 on an out-of-range page id / bad argument.
+ */
+int mfa_oracle_decode(int B, int H, int D, const uint16_t* q,
+                      const void* k, const void* v, int kv_dtype,
+                      int64_t batch_stride, int64_t token_stride,
+                      const int32_t* page_table, int max_pages, int page_size, int num_pages,
+                      const int32_t* seq_lens, double scale, double k_scale, double v_scale,
+                      const int32_t* sel_b, const int32_t* sel_h, int nsel,
+                      double* out, double* lse) {
+    int npairs = sel_b ? nsel : B * H;
+    int bad = 0;
+    if (B < 0 || H <= 0 || D <= 0 || npairs < 0) return -1;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int p = 0; p < npairs; ++p) {
+        int b = sel_b ? sel_b[p] : p / H;
+        int h = sel_b ? sel_h[p] : p % H;
+        double* o = out + (int64_t)p * D;
+        int L = seq_lens[b];
+        if (L <= 0) {
+            for (int i = 0; i < D; ++i) o[i] = 0.0;
+            if (lse) lse[p] = -INFINITY;
+            continue;
+        }
+        double* s = (double*)malloc(sizeof(double) * (size_t)L);
+        double* qv = (double*)malloc(sizeof(double) * (size_t)D);
+        for (int i = 0; i < D; ++i) qv[i] = bf16_bits_to_double(q[((int64_t)b * H + h) * D + i]);
+
+        /* scores */
+        double smax = -INFINITY;
+        for (int t = 0; t < L; ++t) {
+            double acc = 0.0;
+            for (int i = 0; i < D; ++i) {
+                int64_t idx = cache_index(b, t, i, D, batch_stride, token_stride, page_table,
+                                          max_pages, page_size, num_pages);
+                if (idx < 0) { bad = 1; acc = 0.0; break; }
+                acc += qv[i] * (cache_elem(k, kv_dtype, idx) * k_scale);
+            }
+            s[t] = scale * acc;
+            if (s[t] > smax) smax = s[t];
+        }
+        /* softmax denominator */
+        double denom = 0.0;
+        for (int t = 0; t < L; ++t) denom += exp(s[t] - smax);
+        /* weighted sum of value rows */
+        for (int i = 0; i < D; ++i) o[i] = 0.0;
+        for (int t = 0; t < L; ++t) {
+            double w = exp(s[t] - smax) / denom;
+            for (int i = 0; i < D; ++i) {
+                int64_t idx = cache_index(b, t, i, D, batch_stride, token_stride, page_table,
+                                          max_pages, page_size, num_pages);
+                if (idx < 0) { bad = 1; break; }
+                o[i] += w * (cache_elem(v, kv_dtype, idx) * v_scale);
+            }
+        }
+        if (lse) lse[p] = smax + log(denom);
+        free(s);
+        free(qv);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Split-KV merge (Flash-Decoding, cited on the DeepSeek-V4 page): n partial
+ * results of the same softmax over disjoint token ranges, each normalised within
+ * its own range and carrying its range's log-sum-exp, merge into the result over
+ * the union:
+ *     lse* = max_s lse_s,  w_s = exp(lse_s - lse*),
+ *     out  = sum_s w_s * out_s / sum_s w_s,   lse = lse* + log(sum_s w_s).
+ * parts: [n][D], part_lse: [n]. Ranges whose lse is -inf (empty) carry no weight.
+ */
+void mfa_oracle_combine(int n, int D, const double* parts, const double* part_lse,
+                        double* out, double* lse_out) {
+    double m = -INFINITY;
+    for (int s = 0; s < n; ++s)
+        if (part_lse[s] > m) m = part_lse[s];
+    for (int i = 0; i < D; ++i) out[i] = 0.0;
+    if (m == -INFINITY) {
+        if (lse_out) *lse_out = -INFINITY;
+        return;
+    }
+    double wsum = 0.0;
+    for (int s = 0; s < n; ++s) {
+        double w = exp(part_lse[s] - m);
+        wsum += w;
+        for (int i = 0; i < D; ++i) out[i] += w * parts[(int64_t)s * D + i];
+    }
+    for (int i = 0; i < D; ++i) out[i] /= wsum;
+    if (lse_out) *lse_out = m + log(wsum);
+}
+
+/*
+ * Low-rank query projection: c = x * W_qa ([B][Dm] x [Dm][R]), q = c * W_qb
+ * ([B][R] x [R][N]); all row-major bf16 bits, result q in double [B][N].
+ * The latent c is kept in double (no rounding).
+ */
+void mfa_oracle_query_proj(int B, int Dm, int R, int N, const uint16_t* x,
+                           const uint16_t* w_qa, const uint16_t* w_qb, double* q_out) {
+    double* c = (double*)calloc((size_t)B * R, sizeof(double));
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < R; ++r) {
+        for (int b = 0; b < B; ++b) {
+            double acc = 0.0;
+            for (int k = 0; k < Dm; ++k)
+                acc += bf16_bits_to_double(x[(int64_t)b * Dm + k]) *
+                       bf16_bits_to_double(w_qa[(int64_t)k * R + r]);
+            c[(int64_t)b * R + r] = acc;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        for (int b = 0; b < B; ++b) {
+            double acc = 0.0;
+            for (int r = 0; r < R; ++r)
+                acc += c[(int64_t)b * R + r] * bf16_bits_to_double(w_qb[(int64_t)r * N + n]);
+            q_out[(int64_t)b * N + n] = acc;
+        }
+    }
+    free(c);
+}
+
+/* Number of OpenMP threads a parallel region here would use (1 without OpenMP). */
+int mfa_oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
