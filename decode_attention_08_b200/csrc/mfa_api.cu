@@ -1,0 +1,501 @@
+// mfa_api.cu -- the extern "C" entry points of libmfa.so (declared in
+// include/mfa.h): argument validation, TMA tensor-map encoding, workspace
+// management and kernel launches. No computation happens here.
+
+#include <cstdio>
+#include <cstring>
+#include <initializer_list>
+#include <mutex>
+
+#include "../../include/mfa.h"
+#include "mfa_internal.h"
+
+namespace mfa {
+int decode_smem_bytes();
+cudaError_t launch_decode(bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);
+int qproj_smem_bytes(int n_cols);
+cudaError_t launch_qproj(const CUtensorMap& tw, const CUtensorMap& ta, const QprojParams& p,
+                         int m_tiles, cudaStream_t stream);
+}  // namespace mfa
+
+using namespace mfa;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// ---------------------------------------------------------------------------
+// device facts and the driver's tensor-map encoder
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+  bool ok = false;
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int current_device(DeviceInfo* info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MFA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ok) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MFA_ERR_CUDA;
+    d.sms = prop.multiProcessorCount;
+    d.cc_major = prop.major;
+    d.cc_minor = prop.minor;
+    d.ok = true;
+  }
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return MFA_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *info = d;
+  if (d.cc_major != 10 || d.cc_minor != 0) return MFA_ERR_UNSUPPORTED;
+  return MFA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// descriptor checks
+// ---------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_size(int dtype) {
+  switch (dtype) {
+    case MFA_BF16: return 2;
+    case MFA_F32: return 4;
+    case MFA_FP8_E4M3: return 1;
+    case MFA_I32: return 4;
+    default: return 0;
+  }
+}
+
+bool well_formed(const mfa_tensor* t, int ndim) {
+  if (!t || !t->data || t->ndim != ndim || elem_size(t->dtype) == 0) return false;
+  for (int i = 0; i < ndim; ++i)
+    if (t->shape[i] < 0 || t->stride[i] < 0) return false;
+  return true;
+}
+
+CUresult encode_3d(CUtensorMap* map, CUtensorMapDataType type, int esize, const void* base,
+                   uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_elems, uint64_t s2_elems,
+                   uint32_t b0, uint32_t b1) {
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1_elems * esize, s2_elems * esize};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+CUresult encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t row_stride_elems, uint32_t b0, uint32_t b1) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_elems * 2};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// ---------------------------------------------------------------------------
+// per-device cached workspaces of the plain entry points
+// ---------------------------------------------------------------------------
+struct CachedWs {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+CachedWs g_ws_decode[kMaxDevices], g_ws_qproj[kMaxDevices];
+
+int cached_workspace(CachedWs* table, size_t need, bool zero, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MFA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  CachedWs& w = table[dev];
+  if (w.bytes < need) {
+    if (w.ptr) {
+      cudaDeviceSynchronize();
+      cudaFree(w.ptr);
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    void* p = nullptr;
+    if (cudaMalloc(&p, need) != cudaSuccess) return MFA_ERR_CUDA;
+    if (zero && cudaMemset(p, 0, need) != cudaSuccess) {
+      cudaFree(p);
+      return MFA_ERR_CUDA;
+    }
+    w.ptr = p;
+    w.bytes = need;
+  }
+  *out = w.ptr;
+  return MFA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct DecodeWsLayout {
+  size_t o_off, lse_off, prefix_off, total;
+  int slots;
+};
+
+DecodeWsLayout decode_ws_layout(int batch, int num_splits, int grid) {
+  DecodeWsLayout l;
+  l.slots = num_splits == 0 ? 2 * grid : batch * num_splits;
+  l.o_off = 0;
+  l.lse_off = align256(l.o_off + static_cast<size_t>(l.slots) * kPartialFloats * sizeof(float));
+  l.prefix_off = align256(l.lse_off + static_cast<size_t>(l.slots) * kHeads * sizeof(float));
+  l.total = align256(l.prefix_off + static_cast<size_t>(batch + 1) * sizeof(int));
+  return l;
+}
+
+constexpr int kMaxSplits = 1024;
+
+int decode_grid(const DeviceInfo& d, int batch, int num_splits) {
+  if (num_splits == 0) return d.sms;
+  const long long units = static_cast<long long>(batch) * num_splits;
+  return static_cast<int>(units < d.sms ? units : d.sms);
+}
+
+// ---------------------------------------------------------------------------
+// query projection workspace: fp32 partials, counters, interleaved latent
+// ---------------------------------------------------------------------------
+struct QprojWsLayout {
+  size_t part_off, cnt_off, lat_off, total;
+  int splits;
+};
+
+QprojWsLayout qproj_ws_layout(int batch, int dm, int rank, int sms) {
+  QprojWsLayout l;
+  const int k_blocks = dm / 64;
+  const int m_tiles = rank / 128;
+  int splits = m_tiles > 0 ? sms / m_tiles : 1;
+  if (splits < 1) splits = 1;
+  if (splits > k_blocks) splits = k_blocks;
+  l.splits = splits;
+  l.part_off = 0;
+  l.cnt_off = align256(static_cast<size_t>(splits) * batch * rank * sizeof(float));
+  l.lat_off = align256(l.cnt_off + static_cast<size_t>(m_tiles) * sizeof(int));
+  l.total = align256(l.lat_off + static_cast<size_t>(2 * batch) * rank * 2);
+  return l;
+}
+
+}  // namespace
+
+// ===========================================================================
+// public entry points
+// ===========================================================================
+extern "C" {
+
+const char* mfa_error_string(int code) {
+  switch (code) {
+    case MFA_OK: return "MFA_OK";
+    case MFA_ERR_INVALID_ARG: return "MFA_ERR_INVALID_ARG: invalid argument";
+    case MFA_ERR_UNSUPPORTED: return "MFA_ERR_UNSUPPORTED: unsupported shape, dtype or device";
+    case MFA_ERR_CUDA: return "MFA_ERR_CUDA: CUDA call or kernel launch failed";
+    case MFA_ERR_WORKSPACE: return "MFA_ERR_WORKSPACE: workspace missing or too small";
+    case MFA_ERR_BAD_INDEX: return "MFA_ERR_BAD_INDEX: page id or sequence length out of range";
+    case MFA_ERR_TIMEOUT: return "MFA_ERR_TIMEOUT: an in-kernel wait exceeded its time limit";
+    default: return "unknown mfa status code";
+  }
+}
+
+int mfa_version(void) { return 100; }
+
+size_t mfa_decode_workspace_size(int batch, int num_splits) {
+  if (batch <= 0 || num_splits < 0 || num_splits > kMaxSplits) return 0;
+  DeviceInfo d;
+  const int rc = current_device(&d);
+  if (rc != MFA_OK && rc != MFA_ERR_UNSUPPORTED) return 0;
+  return decode_ws_layout(batch, num_splits, decode_grid(d, batch, num_splits)).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validates every argument (host only, no CUDA call) and, unless
+// validate_only, encodes the tensor maps and launches.
+int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor* v_cache,
+                const mfa_tensor* page_table, const mfa_tensor* seq_lens, mfa_tensor* out,
+                float softmax_scale, int kv_dtype, float k_scale, float v_scale, int num_splits,
+                mfa_tensor* lse_out, void* workspace, size_t workspace_bytes, mfa_stream_t stream,
+                bool validate_only) {
+  // ---- shapes and dtypes ----
+  if (!well_formed(q, 3) || !well_formed(k_cache, 3) || !well_formed(v_cache, 3) ||
+      !well_formed(seq_lens, 1) || !well_formed(out, 3))
+    return MFA_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale) || !(k_scale == k_scale) || !(v_scale == v_scale))
+    return MFA_ERR_INVALID_ARG;
+  if (num_splits < 0 || num_splits > kMaxSplits) return MFA_ERR_INVALID_ARG;
+  const int64_t B = q->shape[0];
+  if (B <= 0 || B > (1 << 20)) return MFA_ERR_INVALID_ARG;
+  if (q->dtype != MFA_BF16) return MFA_ERR_INVALID_ARG;
+  if (q->shape[1] != kHeads || q->shape[2] != kDim) return MFA_ERR_UNSUPPORTED;
+  if (q->stride[2] != 1 || q->stride[1] % 8 || q->stride[0] % 8) return MFA_ERR_INVALID_ARG;
+  if (kv_dtype != MFA_BF16 && kv_dtype != MFA_FP8_E4M3) return MFA_ERR_INVALID_ARG;
+  if (k_cache->dtype != kv_dtype || v_cache->dtype != kv_dtype) return MFA_ERR_INVALID_ARG;
+  if (kv_dtype == MFA_FP8_E4M3) return MFA_ERR_UNSUPPORTED;  // FP8 path: see decode_fp8
+  if (kv_dtype == MFA_BF16 && (k_scale != 1.f || v_scale != 1.f)) return MFA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (k_cache->shape[i] != v_cache->shape[i]) return MFA_ERR_INVALID_ARG;
+  if (k_cache->shape[2] != kDim) return MFA_ERR_UNSUPPORTED;
+  const int esz = elem_size(kv_dtype);
+  for (const mfa_tensor* t : {k_cache, v_cache}) {
+    if (t->stride[2] != 1 || (t->stride[1] * esz) % 16 || (t->stride[0] * esz) % 16 ||
+        !aligned16(t->data))
+      return MFA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q->data)) return MFA_ERR_INVALID_ARG;
+  if (seq_lens->dtype != MFA_I32 || seq_lens->shape[0] != B || seq_lens->stride[0] != 1)
+    return MFA_ERR_INVALID_ARG;
+  if (out->dtype != MFA_BF16 && out->dtype != MFA_F32) return MFA_ERR_INVALID_ARG;
+  if (out->shape[0] != B || out->shape[1] != kHeads || out->shape[2] != kDim ||
+      out->stride[2] != 1)
+    return MFA_ERR_INVALID_ARG;
+  if (lse_out) {
+    if (!well_formed(lse_out, 2) || lse_out->dtype != MFA_F32 || lse_out->shape[0] != B ||
+        lse_out->shape[1] != kHeads || lse_out->stride[1] != 1)
+      return MFA_ERR_INVALID_ARG;
+  }
+  const bool paged = page_table != nullptr;
+  int page_size = 0, max_pages = 0, num_pages = 0;
+  int64_t cap = 0;
+  if (paged) {
+    if (!well_formed(page_table, 2) || page_table->dtype != MFA_I32 ||
+        page_table->shape[0] != B || page_table->stride[1] != 1)
+      return MFA_ERR_INVALID_ARG;
+    page_size = static_cast<int>(k_cache->shape[1]);
+    if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128 &&
+        page_size != 256)
+      return MFA_ERR_UNSUPPORTED;
+    if (k_cache->shape[0] <= 0 || k_cache->shape[0] > (1ll << 31) - 1) return MFA_ERR_INVALID_ARG;
+    num_pages = static_cast<int>(k_cache->shape[0]);
+    if (page_table->shape[1] <= 0 || page_table->shape[1] > (1 << 24)) return MFA_ERR_INVALID_ARG;
+    max_pages = static_cast<int>(page_table->shape[1]);
+    cap = static_cast<int64_t>(max_pages) * page_size;
+    if (k_cache->stride[1] != kDim || v_cache->stride[1] != kDim) return MFA_ERR_INVALID_ARG;
+  } else {
+    if (k_cache->shape[0] != B) return MFA_ERR_INVALID_ARG;
+    cap = k_cache->shape[1];
+  }
+  if (cap > (1 << 30)) return MFA_ERR_UNSUPPORTED;
+  if (validate_only) return MFA_OK;
+
+  DeviceInfo dev;
+  int rc = current_device(&dev);
+  if (rc != MFA_OK) return rc;
+  const int grid = decode_grid(dev, static_cast<int>(B), num_splits);
+  const DecodeWsLayout wl = decode_ws_layout(static_cast<int>(B), num_splits, grid);
+  if (!workspace || workspace_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return MFA_ERR_WORKSPACE;
+
+  // ---- tensor maps ----
+  CUtensorMap tq, tk, tv;
+  if (encode_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q->data, kDim, kHeads, B, q->stride[1],
+                q->stride[0], 64, 64) != CUDA_SUCCESS)
+    return MFA_ERR_INVALID_ARG;
+  const int rows = paged ? (page_size < kTile ? page_size : kTile) : kTile;
+  const uint64_t d1 = paged ? static_cast<uint64_t>(page_size) : static_cast<uint64_t>(cap);
+  const uint64_t d2 = paged ? static_cast<uint64_t>(num_pages) : static_cast<uint64_t>(B);
+  if (cap == 0 && !paged) {
+    // a zero-length cache: nothing is ever loaded, but a map needs extent >= 1
+  }
+  const uint64_t d1s = d1 > 0 ? d1 : 1;
+  if (encode_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_cache->data, kDim, d1s, d2,
+                k_cache->stride[1], k_cache->stride[0], 64, rows) != CUDA_SUCCESS ||
+      encode_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v_cache->data, kDim, d1s, d2,
+                v_cache->stride[1], v_cache->stride[0], 64, rows) != CUDA_SUCCESS)
+    return MFA_ERR_INVALID_ARG;
+
+  DecodeParams p;
+  std::memset(&p, 0, sizeof p);
+  p.seq_lens = static_cast<const int*>(seq_lens->data);
+  p.batch = static_cast<int>(B);
+  p.cap_tokens = static_cast<int>(cap);
+  p.paged = paged;
+  p.page_size = page_size;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.page_table = paged ? static_cast<const int*>(page_table->data) : nullptr;
+  p.pt_stride = paged ? page_table->stride[0] : 0;
+  p.num_splits = num_splits;
+  p.grid = grid;
+  p.score_log2 = softmax_scale * k_scale * 1.4426950408889634f;
+  p.out_scale = v_scale;
+  p.out = out->data;
+  p.out_f32 = out->dtype == MFA_F32;
+  p.out_sb = out->stride[0];
+  p.out_sh = out->stride[1];
+  p.lse_out = lse_out ? static_cast<float*>(lse_out->data) : nullptr;
+  p.lse_sb = lse_out ? lse_out->stride[0] : 0;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+  p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
+  p.ws_prefix = reinterpret_cast<int*>(ws + wl.prefix_off);
+
+  const cudaError_t err = launch_decode(paged, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mfa_decode_attention_ex(const mfa_tensor* q, const mfa_tensor* k_cache,
+                            const mfa_tensor* v_cache, const mfa_tensor* page_table,
+                            const mfa_tensor* seq_lens, mfa_tensor* out, float softmax_scale,
+                            int kv_dtype, float k_scale, float v_scale, int num_splits,
+                            mfa_tensor* lse_out, void* workspace, size_t workspace_bytes,
+                            mfa_stream_t stream) {
+  return decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, kv_dtype,
+                     k_scale, v_scale, num_splits, lse_out, workspace, workspace_bytes, stream,
+                     false);
+}
+
+int mfa_decode_attention(const mfa_tensor* q, const mfa_tensor* k_cache,
+                         const mfa_tensor* v_cache, const mfa_tensor* page_table,
+                         const mfa_tensor* seq_lens, mfa_tensor* out, float softmax_scale,
+                         int kv_dtype, mfa_stream_t stream) {
+  const int vrc = decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale,
+                              kv_dtype, 1.f, 1.f, 0, nullptr, nullptr, 0, stream, true);
+  if (vrc != MFA_OK) return vrc;
+  const size_t need = mfa_decode_workspace_size(static_cast<int>(q->shape[0]), 0);
+  if (need == 0) return MFA_ERR_CUDA;
+  void* ws = nullptr;
+  const int rc = cached_workspace(g_ws_decode, need, false, &ws);
+  if (rc != MFA_OK) return rc;
+  return mfa_decode_attention_ex(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale,
+                                 kv_dtype, 1.f, 1.f, 0, nullptr, ws, need, stream);
+}
+
+size_t mfa_query_proj_workspace_size(int batch, int dm, int rank) {
+  if (batch <= 0 || dm <= 0 || rank <= 0) return 0;
+  DeviceInfo d;
+  const int rc = current_device(&d);
+  if (rc != MFA_OK && rc != MFA_ERR_UNSUPPORTED) return 0;
+  return qproj_ws_layout(batch, dm, rank, d.sms).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+int qproj_impl(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
+               mfa_tensor* q_out, void* workspace, size_t workspace_bytes, mfa_stream_t stream,
+               bool validate_only) {
+  if (!well_formed(x, 2) || !well_formed(w_qa, 2) || !well_formed(w_qb, 2) ||
+      !well_formed(q_out, 2))
+    return MFA_ERR_INVALID_ARG;
+  for (const mfa_tensor* t : std::initializer_list<const mfa_tensor*>{x, w_qa, w_qb, q_out})
+    if (t->dtype != MFA_BF16 || t->stride[1] != 1 || t->stride[0] % 8 || !aligned16(t->data))
+      return MFA_ERR_INVALID_ARG;
+  const int64_t B = x->shape[0], Dm = x->shape[1], R = w_qa->shape[1], N = w_qb->shape[1];
+  if (w_qa->shape[0] != Dm || w_qb->shape[0] != R || q_out->shape[0] != B || q_out->shape[1] != N)
+    return MFA_ERR_INVALID_ARG;
+  if (B < 1 || B > 128 || Dm % 64 || R % 128 || N % 128 || Dm <= 0 || R <= 0 || N <= 0 ||
+      Dm > (1 << 20) || R > (1 << 20) || N > (1 << 24))
+    return MFA_ERR_UNSUPPORTED;
+  if (validate_only) return MFA_OK;
+
+  DeviceInfo dev;
+  int rc = current_device(&dev);
+  if (rc != MFA_OK) return rc;
+  const QprojWsLayout wl = qproj_ws_layout(static_cast<int>(B), static_cast<int>(Dm),
+                                           static_cast<int>(R), dev.sms);
+  if (!workspace || workspace_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return MFA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* latent = reinterpret_cast<__nv_bfloat16*>(ws + wl.lat_off);
+
+  const int n1 = static_cast<int>((B + 15) / 16 * 16);
+  const int n2 = static_cast<int>((2 * B + 15) / 16 * 16);
+  CUtensorMap tw1, tx, tw2, tl;
+  if (encode_2d(&tw1, w_qa->data, R, Dm, w_qa->stride[0], 64, 64) != CUDA_SUCCESS ||
+      encode_2d(&tx, x->data, Dm, B, x->stride[0], 64, n1) != CUDA_SUCCESS ||
+      encode_2d(&tw2, w_qb->data, N, R, w_qb->stride[0], 64, 64) != CUDA_SUCCESS ||
+      encode_2d(&tl, latent, R, 2 * B, R, 64, n2) != CUDA_SUCCESS)
+    return MFA_ERR_INVALID_ARG;
+
+  QprojParams p1;
+  std::memset(&p1, 0, sizeof p1);
+  p1.batch = static_cast<int>(B);
+  p1.k_blocks = static_cast<int>(Dm / 64);
+  p1.m_total = static_cast<int>(R);
+  p1.splits = wl.splits;
+  p1.n_cols = n1;
+  p1.mode = 0;
+  p1.partials = reinterpret_cast<float*>(ws + wl.part_off);
+  p1.counters = reinterpret_cast<int*>(ws + wl.cnt_off);
+  p1.latent = latent;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_qproj(tw1, tx, p1, static_cast<int>(R / 128), st) != cudaSuccess) return MFA_ERR_CUDA;
+
+  QprojParams p2 = p1;
+  p2.k_blocks = static_cast<int>(R / 64);
+  p2.m_total = static_cast<int>(N);
+  p2.splits = 1;
+  p2.n_cols = n2;
+  p2.mode = 1;
+  p2.q_out = static_cast<__nv_bfloat16*>(q_out->data);
+  p2.q_stride = q_out->stride[0];
+  if (launch_qproj(tw2, tl, p2, static_cast<int>(N / 128), st) != cudaSuccess) return MFA_ERR_CUDA;
+  return MFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mfa_query_proj_ex(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
+                      mfa_tensor* q_out, void* workspace, size_t workspace_bytes,
+                      mfa_stream_t stream) {
+  return qproj_impl(x, w_qa, w_qb, q_out, workspace, workspace_bytes, stream, false);
+}
+
+int mfa_query_proj(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
+                   mfa_tensor* q_out, mfa_stream_t stream) {
+  const int vrc = qproj_impl(x, w_qa, w_qb, q_out, nullptr, 0, stream, true);
+  if (vrc != MFA_OK) return vrc;
+  const size_t need = mfa_query_proj_workspace_size(static_cast<int>(x->shape[0]),
+                                                    static_cast<int>(x->shape[1]),
+                                                    static_cast<int>(w_qa->shape[1]));
+  if (need == 0) return MFA_ERR_CUDA;
+  void* ws = nullptr;
+  const int rc = cached_workspace(g_ws_qproj, need, true, &ws);
+  if (rc != MFA_OK) return rc;
+  return mfa_query_proj_ex(x, w_qa, w_qb, q_out, ws, need, stream);
+}
+
+int mfa_read_status(mfa_stream_t stream, int reset, int* status_out) {
+  if (!status_out) return MFA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MFA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_mfa_status, sizeof v) != cudaSuccess) return MFA_ERR_CUDA;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_mfa_status, &zero, sizeof zero) != cudaSuccess) return MFA_ERR_CUDA;
+  }
+  *status_out = v;
+  return MFA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// mfa_internal.h -- parameter blocks shared by the host launchers and the
+// kernels of libmfa.so (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace mfa {
+
+constexpr int kHeads = 64;    // query heads per token
+constexpr int kDim = 256;     // head dimension of q and of the shared K / V heads
+constexpr int kTile = 128;    // cached tokens per tile = MMA M of the score product
+
+// Decode-attention kernel geometry (bf16 cache).
+constexpr int kSlots = 5;                  // TMA ring slots
+constexpr int kSlotBytes = 128 * 128 * 2;  // one tensor, 128 tokens x 128 dims, bf16
+constexpr int kQBytes = kHeads * kDim * 2;
+constexpr int kPBytes = kTile * kHeads * 2;
+constexpr int kDecodeThreads = 256;        // 8 warps
+constexpr int kTmemCols = 256;             // S0 | S1 | O_lo | O_hi, 64 columns each
+
+// One partial (split) result: O [64][256] f32 normalised over its range.
+constexpr size_t kPartialFloats = static_cast<size_t>(kHeads) * kDim;
+
+struct DecodeParams {
+  const int* seq_lens;
+  int batch;
+  int cap_tokens;       // largest valid sequence length
+  int paged;
+  int page_size;
+  int max_pages;
+  int num_pages;
+  const int* page_table;
+  int64_t pt_stride;    // elements between page-table rows
+  int num_splits;       // 0: balanced plan over grid; s > 0: s units per sequence
+  int grid;             // CTAs of the attention kernel (the plan depends on it)
+  float score_log2;     // softmax_scale * k_scale * log2(e)
+  float out_scale;      // v_scale
+  void* out;
+  int out_f32;
+  int64_t out_sb, out_sh;  // out strides (elements) of batch and head; d stride 1
+  float* lse_out;          // nullable [B][64]
+  int64_t lse_sb;
+  float* ws_o;             // [slots][64][256]
+  float* ws_lse;           // [slots][64]
+  int* ws_prefix;          // [B + 1] tile prefix (balanced plan only)
+};
+
+struct QprojParams {
+  int batch;
+  int k_blocks;          // contraction length / 64
+  int m_total;           // output features of this GEMM
+  int splits;            // split-K factor (first GEMM)
+  int n_cols;            // MMA N (16..256)
+  int mode;              // 0: latent GEMM (split-K, fp32 partials, hi/lo latent), 1: up-projection
+  float* partials;       // [splits][batch][m_total]  (mode 0)
+  int* counters;         // [m_total / 128]           (mode 0)
+  __nv_bfloat16* latent; // [2 * batch][m_total], rows 2j / 2j+1 = high part / residual
+  __nv_bfloat16* q_out;  // (mode 1 output)
+  int64_t q_stride;      // elements between q_out rows
+};
+
+}  // namespace mfa

@@ -1,0 +1,187 @@
+"""Python binding of libmfa.so (C ABI in ``include/mfa.h``).
+
+Argument marshalling only: torch tensors become ``mfa_tensor`` descriptors,
+the current CUDA stream is passed through, and every step of the computation
+runs in the library's kernels. There is no fallback: if ``libmfa.so`` is
+missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmfa.so")
+
+MFA_BF16, MFA_F32, MFA_FP8_E4M3, MFA_I32 = 0, 1, 2, 3
+STATUS = {
+    0: "MFA_OK", 1: "MFA_ERR_INVALID_ARG", 2: "MFA_ERR_UNSUPPORTED", 3: "MFA_ERR_CUDA",
+    4: "MFA_ERR_WORKSPACE", 5: "MFA_ERR_BAD_INDEX", 6: "MFA_ERR_TIMEOUT",
+}
+STATUS_CODES = {v: k for k, v in STATUS.items()}
+H, D = 64, 256
+
+
+class MfaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class MfaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+EXPORTS = ("mfa_decode_attention", "mfa_decode_attention_ex", "mfa_decode_workspace_size",
+           "mfa_query_proj", "mfa_query_proj_ex", "mfa_query_proj_workspace_size",
+           "mfa_read_status", "mfa_error_string", "mfa_version")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m decode_attention_08_b200.build`"
+                    " (there is no CPU fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            P, T = ctypes.c_void_p, ctypes.POINTER(MfaTensor)
+            L.mfa_decode_attention.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, P]
+            L.mfa_decode_attention.restype = ctypes.c_int
+            L.mfa_decode_attention_ex.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int,
+                                                  ctypes.c_float, ctypes.c_float, ctypes.c_int, T,
+                                                  P, ctypes.c_size_t, P]
+            L.mfa_decode_attention_ex.restype = ctypes.c_int
+            L.mfa_decode_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int]
+            L.mfa_decode_workspace_size.restype = ctypes.c_size_t
+            L.mfa_query_proj.argtypes = [T, T, T, T, P]
+            L.mfa_query_proj.restype = ctypes.c_int
+            L.mfa_query_proj_ex.argtypes = [T, T, T, T, P, ctypes.c_size_t, P]
+            L.mfa_query_proj_ex.restype = ctypes.c_int
+            L.mfa_query_proj_workspace_size.argtypes = [ctypes.c_int] * 3
+            L.mfa_query_proj_workspace_size.restype = ctypes.c_size_t
+            L.mfa_read_status.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+            L.mfa_read_status.restype = ctypes.c_int
+            L.mfa_error_string.argtypes = [ctypes.c_int]
+            L.mfa_error_string.restype = ctypes.c_char_p
+            L.mfa_version.argtypes = []
+            L.mfa_version.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+_DTYPES = {torch.bfloat16: MFA_BF16, torch.float32: MFA_F32, torch.uint8: MFA_FP8_E4M3,
+           torch.float8_e4m3fn: MFA_FP8_E4M3, torch.int32: MFA_I32}
+
+
+def describe(t: Optional[torch.Tensor]):
+    """ctypes pointer to an mfa_tensor describing ``t`` (None -> NULL)."""
+    if t is None:
+        return None
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    d = MfaTensor()
+    d.data = t.data_ptr()
+    d.dtype = _DTYPES[t.dtype]
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return ctypes.pointer(d)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise MfaError(rc, what)
+
+
+def _kv_code(kv_dtype) -> int:
+    if kv_dtype in ("bf16", MFA_BF16, torch.bfloat16):
+        return MFA_BF16
+    if kv_dtype in ("e4m3", "fp8", MFA_FP8_E4M3, torch.float8_e4m3fn, torch.uint8):
+        return MFA_FP8_E4M3
+    raise ValueError(f"kv_dtype {kv_dtype!r}")
+
+
+def decode_attention(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale=1.0 / 16,
+                     kv_dtype="bf16", stream=None):
+    """``mfa_decode_attention``: out = softmax(scale q K^T) V per head over each sequence."""
+    rc = lib().mfa_decode_attention(describe(q), describe(k_cache), describe(v_cache),
+                                    describe(page_table), describe(seq_lens), describe(out),
+                                    float(softmax_scale), _kv_code(kv_dtype), _stream(stream))
+    _check(rc, "mfa_decode_attention")
+    return out
+
+
+def decode_workspace_size(batch: int, num_splits: int = 0) -> int:
+    return int(lib().mfa_decode_workspace_size(int(batch), int(num_splits)))
+
+
+def decode_attention_ex(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale=1.0 / 16,
+                        kv_dtype="bf16", k_scale=1.0, v_scale=1.0, num_splits=0, lse_out=None,
+                        workspace: Optional[torch.Tensor] = None, stream=None):
+    """``mfa_decode_attention_ex`` (scales, split control, lse, caller workspace)."""
+    need = decode_workspace_size(q.shape[0], num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib().mfa_decode_attention_ex(
+        describe(q), describe(k_cache), describe(v_cache), describe(page_table),
+        describe(seq_lens), describe(out), float(softmax_scale), _kv_code(kv_dtype),
+        float(k_scale), float(v_scale), int(num_splits), describe(lse_out),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mfa_decode_attention_ex")
+    return out
+
+
+def query_proj(x, w_qa, w_qb, q_out, stream=None):
+    """``mfa_query_proj``: q_out = (x W_qa) W_qb."""
+    rc = lib().mfa_query_proj(describe(x), describe(w_qa), describe(w_qb), describe(q_out),
+                              _stream(stream))
+    _check(rc, "mfa_query_proj")
+    return q_out
+
+
+def query_proj_workspace_size(batch: int, dm: int, rank: int) -> int:
+    return int(lib().mfa_query_proj_workspace_size(int(batch), int(dm), int(rank)))
+
+
+def query_proj_ex(x, w_qa, w_qb, q_out, workspace: torch.Tensor, stream=None):
+    rc = lib().mfa_query_proj_ex(describe(x), describe(w_qa), describe(w_qb), describe(q_out),
+                                 workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mfa_query_proj_ex")
+    return q_out
+
+
+def read_status(stream=None, reset: bool = True) -> int:
+    """Synchronise ``stream`` and read the device status word (0 = no error)."""
+    v = ctypes.c_int(0)
+    _check(lib().mfa_read_status(_stream(stream), int(bool(reset)), ctypes.byref(v)),
+           "mfa_read_status")
+    return v.value
+
+
+def error_string(code: int) -> str:
+    return lib().mfa_error_string(int(code)).decode()
+
+
+def version() -> int:
+    return int(lib().mfa_version())

@@ -1,0 +1,170 @@
+/*
+ * mfa.h -- C ABI of libmfa.so: Multi-Matrix Factorization Attention (MFA) at
+ * decode, and the MFA low-rank query projection, on NVIDIA B200 (sm_100a).
+ *
+ * What the operations are (Step-3 page, "Key points -> Architecture"): each new
+ * token has 64 query heads of dimension 256, produced from the 7168-wide hidden
+ * state through a 2048-wide low-rank bottleneck, and all 64 heads attend over a
+ * single shared key head and a single shared value head of dimension 256 held in
+ * the KV cache. The pages print no formula; the operation implemented is
+ *
+ *     out[b,h,:] = softmax_t( softmax_scale * q[b,h,:] . K_b[t,:] ) V_b[t,:],   t < seq_lens[b]
+ *
+ * with optional lse[b,h] = log sum_t exp(softmax_scale * q[b,h,:] . K_b[t,:]).
+ * An empty sequence (seq_lens[b] == 0) yields zeros and lse = -inf.
+ * K_b/V_b come from a contiguous slab or through a page table (PagedAttention,
+ * cited in the Step-3 page's references). The pages deploy attention in FP8 and
+ * in BF16 (Step-3 page, "Key points -> Throughput" and "Ablations"): the cache
+ * may be bf16 or FP8 E4M3 with per-tensor scales. Long contexts are split over
+ * many CTAs and merged with a log-sum-exp combine (Flash-Decoding, cited on the
+ * DeepSeek-V4 page's reference list).
+ *
+ * Conventions for every entry point:
+ *  - All tensor data pointers are DEVICE pointers on the current CUDA device;
+ *    the mfa_tensor descriptor structs themselves live in host memory and are
+ *    only read during the call. The caller owns every buffer.
+ *  - Strides are in ELEMENTS. The innermost (last) dimension must have stride 1.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronise the host.
+ *  - The return value reports host-detectable errors (bad descriptor, unsupported
+ *    shape, too small workspace) and launch errors. Errors the GPU detects
+ *    (a page id outside the pool, a sequence length outside the cache) are
+ *    recorded in a per-device status word read by mfa_read_status(); outputs of
+ *    the affected call are then unspecified, but no access leaves the buffers
+ *    described by the arguments.
+ *  - H = 64 and head dim = 256 are fixed; other shapes return MFA_ERR_UNSUPPORTED.
+ *  - Requires a device of compute capability 10.0 (B200); otherwise
+ *    MFA_ERR_UNSUPPORTED.
+ */
+#ifndef MFA_H_
+#define MFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mfa_stream_t; /* identical to cudaStream_t */
+
+enum mfa_dtype { MFA_BF16 = 0, MFA_F32 = 1, MFA_FP8_E4M3 = 2, MFA_I32 = 3 };
+
+enum mfa_status {
+  MFA_OK = 0,
+  MFA_ERR_INVALID_ARG = 1,  /* null pointer, wrong rank/dtype, inconsistent shapes, bad stride */
+  MFA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (shape, device) */
+  MFA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a kernel launch failed */
+  MFA_ERR_WORKSPACE = 4,    /* caller workspace missing or too small */
+  MFA_ERR_BAD_INDEX = 5,    /* (status word) page id or sequence length out of range */
+  MFA_ERR_TIMEOUT = 6       /* (status word) a bounded in-kernel wait gave up */
+};
+
+/* A strided view of device memory. ndim in [1, 4]; shape/stride beyond ndim are
+ * ignored. Strides in elements; data aligned to at least 16 bytes. */
+typedef struct {
+  void* data;
+  int32_t dtype;  /* enum mfa_dtype */
+  int32_t ndim;
+  int64_t shape[4];
+  int64_t stride[4];
+} mfa_tensor;
+
+/*
+ * MFA decode attention (the operation above).
+ *
+ *  q          [B, 64, 256] bf16. Head and batch strides multiples of 8 elements.
+ *  k_cache    contiguous: [B, Lmax, 256]; paged: [num_pages, page_size, 256].
+ *             dtype MFA_BF16 or MFA_FP8_E4M3, equal to kv_dtype. Token and
+ *             batch/page strides must be multiples of 16 bytes.
+ *  v_cache    same shape, strides and dtype as k_cache.
+ *  page_table NULL for a contiguous cache. Otherwise [B, max_pages] int32:
+ *             token t of sequence b is row t % page_size of page
+ *             page_table[b][t / page_size]. page_size in {16, 32, 64, 128, 256}.
+ *             Entries past ceil(seq_lens[b] / page_size) are never read.
+ *  seq_lens   [B] int32 on the device. 0 <= seq_lens[b] <= Lmax (contiguous) or
+ *             <= max_pages * page_size (paged). Rows past seq_lens[b] are never
+ *             used, whatever they hold (NaN included).
+ *  out        [B, 64, 256], MFA_BF16 or MFA_F32, any strides (d stride 1).
+ *  softmax_scale  multiplies q.k (1/16 = 1/sqrt(256) in the Step-3 setting).
+ *  kv_dtype   MFA_BF16 or MFA_FP8_E4M3 (then k_scale = v_scale = 1).
+ *
+ * Uses a per-device workspace that the library allocates on the first call on
+ * each device (cudaMalloc; keep that first call outside stream capture) and
+ * reuses afterwards; concurrent calls on different streams share it and must
+ * use mfa_decode_attention_ex with their own workspaces instead.
+ */
+int mfa_decode_attention(const mfa_tensor* q, const mfa_tensor* k_cache,
+                         const mfa_tensor* v_cache, const mfa_tensor* page_table,
+                         const mfa_tensor* seq_lens, mfa_tensor* out, float softmax_scale,
+                         int kv_dtype, mfa_stream_t stream);
+
+/*
+ * As mfa_decode_attention, plus:
+ *  k_scale, v_scale  per-tensor dequantisation scales of an FP8 cache
+ *                    (K = code * k_scale, V = code * v_scale); must be 1 for bf16.
+ *  num_splits        0: balanced split of all (sequence, 128-token tile) work over
+ *                    the GPU's SMs (the default). s > 0: every sequence is cut
+ *                    into s nearly equal token ranges, each its own work unit.
+ *  lse_out           NULL or [B, 64] f32: natural-log log-sum-exp of the scaled
+ *                    scores (-inf for empty sequences).
+ *  workspace         device memory of at least
+ *                    mfa_decode_workspace_size(B, num_splits) bytes, 256-byte
+ *                    aligned. Contents need no initialisation.
+ * Splitting never changes which cached rows contribute; the split plan depends
+ * only on seq_lens, num_splits and the SM count, never on the cache layout, so a
+ * paged and a contiguous cache holding the same rows give bit-identical results.
+ */
+int mfa_decode_attention_ex(const mfa_tensor* q, const mfa_tensor* k_cache,
+                            const mfa_tensor* v_cache, const mfa_tensor* page_table,
+                            const mfa_tensor* seq_lens, mfa_tensor* out, float softmax_scale,
+                            int kv_dtype, float k_scale, float v_scale, int num_splits,
+                            mfa_tensor* lse_out, void* workspace, size_t workspace_bytes,
+                            mfa_stream_t stream);
+
+/* Bytes of workspace mfa_decode_attention_ex needs for `batch` sequences on the
+ * current device with the given num_splits. 0 on error. */
+size_t mfa_decode_workspace_size(int batch, int num_splits);
+
+/*
+ * MFA low-rank query projection (Step-3 page, "Queries pass through a 2048-dim
+ * low-rank bottleneck"): q_out = (x * W_qa) * W_qb, no bias, norm or activation.
+ *
+ *  x      [B, Dm] bf16 (Dm = 7168 in Step-3), row stride multiple of 8 elements.
+ *  w_qa   [Dm, R] bf16 row-major (R = 2048).
+ *  w_qb   [R, N] bf16 row-major (N = 64 * 256 = 16384).
+ *  q_out  [B, N] bf16 (viewable as [B, 64, 256] when N = 16384).
+ * 1 <= B <= 128; Dm, R multiples of 64; N a multiple of 128.
+ * The latent x * W_qa is accumulated in fp32 and carried into the second product
+ * at about 16 significant bits (a bf16 high part plus a bf16 residual); q_out is
+ * rounded once, to bf16.
+ * Uses a per-device cached workspace (allocated on the first call; see above).
+ */
+int mfa_query_proj(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
+                   mfa_tensor* q_out, mfa_stream_t stream);
+
+/* As mfa_query_proj with a caller workspace of at least
+ * mfa_query_proj_workspace_size(B, Dm, R) bytes, 256-byte aligned, that must be
+ * zero-filled before its first use; every call leaves it zero-filled again. */
+int mfa_query_proj_ex(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
+                      mfa_tensor* q_out, void* workspace, size_t workspace_bytes,
+                      mfa_stream_t stream);
+
+size_t mfa_query_proj_workspace_size(int batch, int dm, int rank);
+
+/* Synchronises `stream`, then reads (and, if reset != 0, clears) the current
+ * device's status word: MFA_OK or the first MFA_ERR_BAD_INDEX / MFA_ERR_TIMEOUT
+ * a kernel recorded since the last reset. Returns MFA_OK or MFA_ERR_CUDA. */
+int mfa_read_status(mfa_stream_t stream, int reset, int* status_out);
+
+/* Static, human-readable name of a status code. */
+const char* mfa_error_string(int code);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int mfa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MFA_H_ */
