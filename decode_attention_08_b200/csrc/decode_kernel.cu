@@ -13,28 +13,68 @@
 // softmax is computed online over 128-token tiles (running max with lazy
 // rescaling, running sum), so each K and V row is read from HBM exactly once.
 //
-// CTA = 8 warps, one CTA per SM (persistent):
-//   warp 0  TMA producer for the K/V ring (5 slots x 32 KB)
-//   warp 1  TMEM allocator + single-thread tcgen05.mma issuer
-//   warp 2  TMA producer for q (one 32 KB load per sequence segment)
-//   warp 3  idle
-//   warps 4-7  softmax + epilogue (thread = one token row of S^T, then one
-//              head-dim row of O^T)
+// CTA = 12 warps, one CTA per SM (persistent):
+//   warp 0       TMA producer for the K/V ring (5 slots x 32 KB)
+//   warp 1       TMEM allocator + tcgen05.mma issuer (one lane issues)
+//   warp 2       TMA producer for q (one 32 KB load per sequence segment)
+//   warp 3       idle
+//   warps 4-7    softmax warpgroup 0: heads 0-31  } thread = one token row of S^T,
+//   warps 8-11   softmax warpgroup 1: heads 32-63 } then one head-dim row of O^T
 //
 // Work split (Flash-Decoding, cited on the DeepSeek-V4 page): the (sequence,
 // 128-token tile) pairs of the whole batch are cut into `grid` contiguous,
 // equal ranges ("balanced"), or every sequence into `num_splits` equal ranges.
-// A range that covers a whole sequence writes the final output; otherwise it
-// writes a normalised partial and its log-sum-exp, merged by mfa_combine_kernel.
-// The plan depends only on seq_lens, num_splits and grid, never on whether the
-// cache is paged, so paged and contiguous caches give bit-identical results.
+// A range that covers a whole sequence writes the final output. Otherwise it
+// writes a partial output normalised over its range plus the range's
+// log-sum-exp, and mfa_combine_kernel merges the partials of each split
+// sequence in plan order (Flash-Decoding's log-sum-exp combine). The plan
+// depends only on seq_lens, num_splits and grid, never on whether the cache is
+// paged, so paged and contiguous caches give bit-identical results.
+//
+// Both kernels are launched with programmatic dependent launch: each may start
+// (set up barriers, TMEM, descriptors) while the previous kernel on the stream
+// drains, and waits with griddepcontrol.wait before touching any input or output.
+
+#include <cstddef>
 
 #include "mfa_internal.h"
 #include "sm100.cuh"
 
 namespace mfa {
 
+// Optional pipeline trace (compile with -DMFA_TRACE; off in the library build):
+// clock64() stamps of pipeline events for the first 64 tiles of each CTA.
+#ifdef MFA_TRACE
+constexpr int kTraceKinds = 12, kTraceTiles = 64, kTraceCtas = 160;
+__device__ unsigned long long g_mfa_trace[kTraceCtas * kTraceKinds * kTraceTiles];
+#define MFA_TR(kind, idx)                                                                   \
+  do {                                                                                      \
+    if ((idx) < kTraceTiles && blockIdx.x < kTraceCtas)                                     \
+      g_mfa_trace[(blockIdx.x * kTraceKinds + (kind)) * kTraceTiles + (idx)] = clock64();   \
+  } while (0)
+// absolute (%globaltimer) timeline of both kernels over consecutive calls:
+// [call][kernel 0 attention / 1 combine][cta][start, after dependency wait, end]
+constexpr int kGtCalls = 8, kGtCtas = 1024;
+__device__ unsigned long long g_mfa_gt[kGtCalls * 2 * kGtCtas * 3];
+__device__ int g_mfa_cnt[2 * kGtCtas];  // per (kernel, CTA) call counter
+#define MFA_GT(kernel, cta, what, call)                                                     \
+  do {                                                                                      \
+    if ((call) >= 0 && (call) < kGtCalls && (cta) < kGtCtas)                                \
+      g_mfa_gt[(((call) * 2 + (kernel)) * kGtCtas + (cta)) * 3 + (what)] = global_timer_ns(); \
+  } while (0)
+#else
+#define MFA_GT(kernel, cta, what, call) \
+  do {                                  \
+  } while (0)
+#define MFA_TR(kind, idx) \
+  do {                    \
+  } while (0)
+#endif
+
 namespace {
+
+constexpr int kWG = 2;  // softmax warpgroups
+constexpr int kWGHeads = kHeads / kWG;
 
 // ---------------------------------------------------------------------------
 // shared-memory control block
@@ -44,28 +84,40 @@ struct __align__(16) DecodeCtrl {
   uint64_t slot_full[kSlots], slot_empty[kSlots];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, o_full;
-  uint64_t red_full[2], l_full;
+  uint64_t red_full[kWG][2], l_full[kWG];
   uint64_t drain;
+  long long t0;    // first global tile of this CTA (balanced plan)
+  long long ntot;  // total tiles of the batch (balanced plan)
   uint32_t tmem_base;
   int abort_flag;
   int b_start, off_start, tiles;
-  int scan_warp[8];
-  float red[2][4][kHeads];   // per-warp tile maxima
-  float mv[4][kHeads];       // per-warp copy of the running max in use
-  float cv[4][kHeads];       // per-warp copy of the rescale factors
-  float lred[4][kHeads];     // per-warp partial row sums (epilogue)
+  int scan_warp[kDecodeThreads / 32];
+  int lens[kDecodeThreads];  // validated seq_lens when batch <= kDecodeThreads
+  // vector-loaded (float4): keep 16-byte aligned
+  alignas(16) float red[2][kWG][4][kWGHeads];  // per-warp tile maxima
+  alignas(16) float mv[kWG][4][kWGHeads];      // per-warp copy: running max in use
+  alignas(16) float cv[kWG][4][kWGHeads];      // per-warp copy: rescale factors / out scale
+  alignas(16) float lred[kWG][4][kWGHeads];    // per-warp partial row sums (epilogue)
 };
+static_assert(offsetof(DecodeCtrl, red) % 16 == 0 && offsetof(DecodeCtrl, mv) % 16 == 0 &&
+                  offsetof(DecodeCtrl, cv) % 16 == 0 && offsetof(DecodeCtrl, lred) % 16 == 0,
+              "vector-loaded control arrays must be 16-byte aligned");
 
 constexpr int kSmemQ = 0;
 constexpr int kSmemRing = kSmemQ + kQBytes;
 constexpr int kSmemP = kSmemRing + kSlots * kSlotBytes;
 constexpr int kSmemCtrl = kSmemP + kPBytes;
 constexpr int kSmemBytes = kSmemCtrl + static_cast<int>(sizeof(DecodeCtrl)) + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // TMEM column map.
 constexpr uint32_t kColS = 0;      // two 64-column score buffers
 constexpr uint32_t kColOlo = 128;  // O^T rows 0..127
 constexpr uint32_t kColOhi = 192;  // O^T rows 128..255
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P entries stay <= 2^8
 
 __device__ __forceinline__ int tiles_of(int L) { return (L + kTile - 1) / kTile; }
 
@@ -78,37 +130,54 @@ __device__ __forceinline__ int valid_len(const DecodeParams& p, int b) {
   return L;
 }
 
+// Sequence length: from the block's shared copy when the batch fits in it.
+__device__ __forceinline__ int seq_len(const DecodeParams& p, const int* lens, int b) {
+  return lens ? lens[b] : valid_len(p, b);
+}
+
+// All lanes wait; the outcome is made warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ uint32_t par(uint32_t u) { return u & 1u; }
+
 // ---------------------------------------------------------------------------
 // The per-CTA stream of tiles, walked independently (and identically) by each
 // role.
 // ---------------------------------------------------------------------------
 struct TileInfo {
-  int b;          // sequence
-  int tile;       // tile index within the sequence
-  int L;          // sequence length
-  bool seg_first; // first tile of a segment (run of tiles of one sequence)
-  bool seg_last;  // last tile of a segment
-  bool cta_last;  // last tile this CTA processes
-  int slot;       // partial slot of the segment, -1 when it covers the sequence
+  int b;            // sequence
+  int tile;         // tile index within the sequence
+  int L;            // sequence length
+  bool seg_first;   // first tile of a segment (run of tiles of one sequence)
+  bool seg_last;    // last tile of a segment
+  bool cta_last;    // last tile this CTA processes
+  int slot;         // partial slot of the segment, -1 when it covers the sequence
+  long long gtile;  // global tile index (balanced plan)
 };
 
 struct TileStream {
   const DecodeParams* p;
+  const int* lens;  // shared copy of the lengths, or nullptr
   int cta;
-  // balanced plan
   int b, tile, L, nt, remaining, seg_lo, seg_hi, seg_ord;
-  // fixed-splits plan
+  long long gtile;
   int unit, unit_hi;
 
-  __device__ void init(const DecodeParams& prm, int b_start, int off_start, int tiles) {
+  __device__ void init(const DecodeParams& prm, const int* lens_, int b_start, int off_start,
+                       int tiles, long long t0) {
     p = &prm;
+    lens = lens_;
     cta = blockIdx.x;
     seg_ord = 0;
+    gtile = t0;
     if (prm.num_splits == 0) {
       remaining = tiles;
       if (remaining > 0) {
         b = b_start;
-        L = valid_len(prm, b);
+        L = seq_len(prm, lens, b);
         nt = tiles_of(L);
         tile = off_start;
         seg_lo = tile;
@@ -128,7 +197,7 @@ struct TileStream {
     for (unit += p->grid; unit < nunits; unit += p->grid) {
       b = unit / s;
       const int j = unit % s;
-      L = valid_len(*p, b);
+      L = seq_len(*p, lens, b);
       nt = tiles_of(L);
       const int lo = static_cast<int>((static_cast<long long>(j) * nt) / s);
       const int hi = static_cast<int>((static_cast<long long>(j + 1) * nt) / s);
@@ -151,16 +220,18 @@ struct TileStream {
     t.L = L;
     t.seg_first = (tile == seg_lo);
     t.seg_last = (tile == seg_hi - 1);
+    t.gtile = gtile;
     const bool complete = (seg_lo == 0 && seg_hi == nt);
     if (p->num_splits == 0) {
       t.slot = complete ? -1 : (2 * cta + (seg_ord == 0 ? 0 : 1));
       ++tile;
+      ++gtile;
       --remaining;
       t.cta_last = (remaining == 0);
       if (remaining > 0 && tile == nt) {
         do {
           ++b;
-          L = valid_len(*p, b);
+          L = seq_len(*p, lens, b);
           nt = tiles_of(L);
         } while (nt == 0);
         tile = 0;
@@ -179,10 +250,60 @@ struct TileStream {
 };
 
 // ---------------------------------------------------------------------------
-// Block-wide plan: total tiles, this CTA's tile range and its first sequence.
-// CTA 0 also stores the per-sequence tile prefix for the combine kernel.
+// The partial slots of a split sequence, in plan order.
 // ---------------------------------------------------------------------------
-__device__ int block_inclusive_scan(int v, int* warp_sums) {
+struct SplitList {
+  int mode;  // 0 balanced, s > 0 fixed
+  long long N, G, S;
+  int c_first, first_slot;
+  bool dense;  // balanced plan with at least one tile per CTA
+  int b, nt;
+  int count;  // candidates in plan order; slot(i) may be -1 (empty range, fixed plan)
+
+  // balanced plan: the sequence's tiles are [S, S + ntiles) in the global order;
+  // CTA c owns tiles [cN/G, (c+1)N/G), so tile t belongs to CTA ((t+1)G - 1) / N.
+  __device__ void init_balanced(long long S_, int ntiles, long long Ntot, long long grid) {
+    mode = 0;
+    N = Ntot;
+    G = grid;
+    S = S_;
+    nt = ntiles;
+    dense = N >= G;
+    c_first = static_cast<int>(((S + 1) * G - 1) / N);
+    const int c_last = static_cast<int>(((S + ntiles) * G - 1) / N);
+    const long long start_first = (static_cast<long long>(c_first) * N) / G;
+    first_slot = (start_first < S) ? 2 * c_first + 1 : 2 * c_first;
+    // with N >= G every CTA owns >= 1 tile; otherwise every CTA owns <= 1 tile
+    count = dense ? c_last - c_first + 1 : ntiles;
+  }
+  __device__ void init_fixed(int seq, int ntiles, int s) {
+    mode = s;
+    b = seq;
+    nt = ntiles;
+    count = s;
+  }
+  __device__ int slot(int i) const {
+    if (mode == 0) {
+      if (i == 0) return first_slot;
+      const long long cc = dense ? c_first + i : ((S + i + 1) * G - 1) / N;
+      return static_cast<int>(2 * cc);
+    }
+    const int lo = static_cast<int>((static_cast<long long>(i) * nt) / mode);
+    const int hi = static_cast<int>((static_cast<long long>(i + 1) * nt) / mode);
+    return hi > lo ? b * mode + i : -1;
+  }
+  __device__ int nonempty() const {
+    if (mode == 0) return count;
+    int n = 0;
+    for (int i = 0; i < count; ++i) n += slot(i) >= 0;
+    return n;
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Block-wide plan: total tiles, this CTA's tile range and its first sequence.
+// ---------------------------------------------------------------------------
+__device__ int block_inclusive_scan(int v, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -191,69 +312,95 @@ __device__ int block_inclusive_scan(int v, int* warp_sums) {
   }
   if (lane == 31) warp_sums[warp] = v;
   __syncthreads();
-  int add = 0;
+  int add = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < kDecodeThreads / 32; ++w)
+  for (int w = 0; w < kDecodeThreads / 32; ++w) {
     if (w < warp) add += warp_sums[w];
-  v += add;
+    tot += warp_sums[w];
+  }
   __syncthreads();
-  return v;
+  *total = tot;
+  return v + add;
 }
 
-__device__ void balanced_plan(const DecodeParams& p, DecodeCtrl& c) {
+// Reads and validates the lengths once; when the batch fits (B <= threads)
+// they stay in shared memory for every role.
+__device__ void load_lengths(const DecodeParams& p, DecodeCtrl& c) {
+  if (p.batch <= kDecodeThreads && threadIdx.x < p.batch) c.lens[threadIdx.x] = valid_len(p, threadIdx.x);
+}
+
+__device__ void balanced_plan(const DecodeParams& p, DecodeCtrl& c, const int* lens) {
   const int tid = threadIdx.x;
-  // pass 1: total number of tiles
   long long total = 0;
-  for (int base = 0; base < p.batch; base += kDecodeThreads) {
-    const int b = base + tid;
-    const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
-    const int incl = block_inclusive_scan(n, c.scan_warp);
-    // the block's last thread holds the chunk total
-    __shared__ int s_chunk;
-    if (tid == kDecodeThreads - 1) s_chunk = incl;
-    __syncthreads();
-    total += s_chunk;
-    __syncthreads();
+  long long t0 = 0;
+  bool located = false;
+  if (lens) {
+    // single pass: the whole batch is one chunk
+    const int n = tid < p.batch ? tiles_of(lens[tid]) : 0;
+    int chunk;
+    const int incl = block_inclusive_scan(n, c.scan_warp, &chunk);
+    total = chunk;
+    const long long G = p.grid;
+    t0 = (static_cast<long long>(blockIdx.x) * total) / G;
+    const long long excl = incl - n;
+    if (tid < p.batch && n > 0 && excl <= t0 && t0 < excl + n) {
+      c.b_start = tid;
+      c.off_start = static_cast<int>(t0 - excl);
+    }
+    if (blockIdx.x == 0) {  // the combine kernel's view of the plan
+      if (tid < p.batch) p.ws_prefix[tid] = static_cast<int>(excl);
+      if (tid == 0) p.ws_prefix[p.batch] = static_cast<int>(total);
+    }
+    located = true;
+  } else {
+    for (int base = 0; base < p.batch; base += kDecodeThreads) {
+      const int b = base + tid;
+      const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
+      int chunk;
+      block_inclusive_scan(n, c.scan_warp, &chunk);
+      total += chunk;
+    }
+    t0 = (static_cast<long long>(blockIdx.x) * total) / p.grid;
   }
-  const long long G = p.grid;
-  const long long t0 = (static_cast<long long>(blockIdx.x) * total) / G;
-  const long long t1 = (static_cast<long long>(blockIdx.x + 1) * total) / G;
+  const long long t1 = (static_cast<long long>(blockIdx.x + 1) * total) / p.grid;
   if (tid == 0) {
     c.tiles = static_cast<int>(t1 - t0);
-    c.b_start = 0;
-    c.off_start = 0;
+    c.t0 = t0;
+    c.ntot = total;
   }
-  // pass 2: locate tile t0; CTA 0 writes the prefix
-  long long run = 0;
-  for (int base = 0; base < p.batch; base += kDecodeThreads) {
-    const int b = base + tid;
-    const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
-    const int incl = block_inclusive_scan(n, c.scan_warp);
-    const long long excl = run + incl - n;
-    if (b < p.batch) {
-      if (blockIdx.x == 0 && p.ws_prefix) p.ws_prefix[b] = static_cast<int>(excl);
-      if (n > 0 && excl <= t0 && t0 < excl + n) {
+  if (!located) {
+    long long run = 0;
+    for (int base = 0; base < p.batch && (run <= t0 || blockIdx.x == 0); base += kDecodeThreads) {
+      const int b = base + tid;
+      const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
+      int chunk;
+      const int incl = block_inclusive_scan(n, c.scan_warp, &chunk);
+      const long long excl = run + incl - n;
+      if (b < p.batch && n > 0 && excl <= t0 && t0 < excl + n) {
         c.b_start = b;
         c.off_start = static_cast<int>(t0 - excl);
       }
+      if (blockIdx.x == 0 && b < p.batch) p.ws_prefix[b] = static_cast<int>(excl);
+      run += chunk;
     }
-    __shared__ int s_chunk2;
-    if (tid == kDecodeThreads - 1) s_chunk2 = incl;
-    __syncthreads();
-    run += s_chunk2;
-    __syncthreads();
+    if (blockIdx.x == 0 && tid == 0) p.ws_prefix[p.batch] = static_cast<int>(total);
   }
-  if (blockIdx.x == 0 && tid == 0 && p.ws_prefix) p.ws_prefix[p.batch] = static_cast<int>(total);
   __syncthreads();
 }
 
+__device__ __forceinline__ void store_out(const DecodeParams& p, int b, int h, int d, float v) {
+  if (p.out_f32)
+    static_cast<float*>(p.out)[b * p.out_sb + h * p.out_sh + d] = v;
+  else
+    static_cast<__nv_bfloat16*>(p.out)[b * p.out_sb + h * p.out_sh + d] = __float2bfloat16_rn(v);
+}
+
 // ---------------------------------------------------------------------------
-// warp-level "reduce-scatter" over the 32 rows a warp holds: on entry each lane
-// has 64 per-head values of its own row; on exit lane l holds, in v[0] and v[1],
-// the reduction over all 32 lanes for heads 2l and 2l+1.
+// warp-level "reduce-scatter": on entry each lane has 32 per-head values of its
+// own row; on exit lane l holds the reduction over all 32 lanes for head l.
 // ---------------------------------------------------------------------------
 template <bool kMax, int N, int MASK>
-__device__ __forceinline__ void rs_step(float (&v)[64], int lane) {
+__device__ __forceinline__ void rs_step(float (&v)[kWGHeads], int lane) {
   const bool upper = (lane & MASK) != 0;
 #pragma unroll
   for (int i = 0; i < N / 2; ++i) {
@@ -265,16 +412,14 @@ __device__ __forceinline__ void rs_step(float (&v)[64], int lane) {
 }
 
 template <bool kMax>
-__device__ __forceinline__ void reduce_scatter64(float (&v)[64], int lane) {
-  rs_step<kMax, 64, 16>(v, lane);
-  rs_step<kMax, 32, 8>(v, lane);
-  rs_step<kMax, 16, 4>(v, lane);
-  rs_step<kMax, 8, 2>(v, lane);
-  rs_step<kMax, 4, 1>(v, lane);
+__device__ __forceinline__ float reduce_scatter32(float (&v)[kWGHeads], int lane) {
+  rs_step<kMax, 32, 16>(v, lane);
+  rs_step<kMax, 16, 8>(v, lane);
+  rs_step<kMax, 8, 4>(v, lane);
+  rs_step<kMax, 4, 2>(v, lane);
+  rs_step<kMax, 2, 1>(v, lane);
+  return v[0];
 }
-
-// Softmax-side parity helper: phase parity of the u-th completion.
-__device__ __forceinline__ uint32_t par(uint32_t u) { return u & 1u; }
 
 // Index, in producer order, of the first (lo) ring item holding V of the CTA's
 // j-th tile: items go K0 | K1 V0 | K2 V1 | ... | K(T-1) V(T-2) | V(T-1), two
@@ -282,10 +427,6 @@ __device__ __forceinline__ uint32_t par(uint32_t u) { return u & 1u; }
 __device__ __forceinline__ uint32_t v_item(uint32_t j, bool cta_last) {
   return cta_last ? 4u * j + 2u : 4u * j + 4u;
 }
-
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: P entries stay <= 2^8
 
 }  // namespace
 
@@ -309,20 +450,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- plan --------------------------------------------------------------
-  if (p.num_splits == 0) {
-    balanced_plan(p, c);
-    if (c.tiles == 0) return;
-  } else {
-    if (static_cast<int>(blockIdx.x) >= p.batch * p.num_splits) return;
-    if (tid == 0) {
-      c.tiles = -1;
-      c.b_start = 0;
-      c.off_start = 0;
-    }
-  }
+  if (tid == 0) MFA_TR(9, 0);
+#ifdef MFA_TRACE
+  const unsigned long long gt_start = global_timer_ns();
+#endif
+  griddep_launch_dependents();
 
-  // ---- setup -------------------------------------------------------------
+  // ---- setup (independent of the previous kernel's results) ----------------
   if (tid == 0) {
     mbar_init(&c.q_full, 1);
     mbar_init(&c.q_empty, 1);
@@ -332,14 +466,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.s_full[i], 1);
-      mbar_init(&c.s_empty[i], 4);
-      mbar_init(&c.red_full[i], 4);
+      mbar_init(&c.s_empty[i], 4 * kWG);
     }
-    mbar_init(&c.p_full, 4);
+    for (int w = 0; w < kWG; ++w) {
+      mbar_init(&c.red_full[w][0], 4);
+      mbar_init(&c.red_full[w][1], 4);
+      mbar_init(&c.l_full[w], 4);
+    }
+    mbar_init(&c.p_full, 4 * kWG);
     mbar_init(&c.o_full, 1);
-    mbar_init(&c.l_full, 4);
     mbar_init(&c.drain, 1);
     c.abort_flag = 0;
+    c.b_start = 0;
+    c.off_start = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -351,6 +490,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+
+  // ---- plan (reads seq_lens: after the previous kernel has completed) -----
+  griddep_wait();
+#ifdef MFA_TRACE
+  const int gt_call = blockIdx.x < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[blockIdx.x]) : -1;
+  if (tid == 0) {
+    MFA_GT(0, blockIdx.x, 1, gt_call);
+    if (gt_call >= 0 && gt_call < kGtCalls && blockIdx.x < kGtCtas)
+      g_mfa_gt[((gt_call * 2) * kGtCtas + blockIdx.x) * 3] = gt_start;
+  }
+#endif
+  const int* lens_s = p.batch <= kDecodeThreads ? c.lens : nullptr;
+  load_lengths(p, c);
+  __syncthreads();
+  if (p.num_splits == 0) {
+    balanced_plan(p, c, lens_s);  // ends with __syncthreads
+  } else if (tid == 0) {
+    c.tiles = static_cast<int>(blockIdx.x) < p.batch * p.num_splits ? -1 : 0;
+    c.t0 = 0;
+    c.ntot = 0;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -358,19 +518,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   volatile int* abort_flag = &c.abort_flag;
   const uint32_t tmem = c.tmem_base;
 
-  if (warp == 0) {
+  if (c.tiles == 0) {
+    // no work for this CTA
+  } else if (warp == 0) {
     // ======================= K/V producer ===================================
-    if (lane == 0) {
-      const uint64_t policy = l2_policy_evict_first();
-      TileStream ks, vs;
-      ks.init(p, c.b_start, c.off_start, c.tiles);
-      vs.init(p, c.b_start, c.off_start, c.tiles);
-      uint32_t item = 0;
-      bool ok = true;
-      auto load = [&](const TileInfo& t, const CUtensorMap* map) -> bool {
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t slot = item % kSlots;
-          if (!mbar_wait(&c.slot_empty[slot], par(item / kSlots) ^ 1u, abort_flag)) return false;
+    const uint64_t policy = l2_policy_evict_first();
+    TileStream ks, vs;
+    ks.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    vs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    uint32_t item = 0;
+    int ntr[2] = {0, 0};
+    auto load = [&](const TileInfo& t, const CUtensorMap* map) -> bool {
+      const int kind = (map == &tm_k) ? 0 : 1;
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t slot = item % kSlots;
+        if (!warp_wait(&c.slot_empty[slot], par(item / kSlots) ^ 1u, abort_flag)) return false;
+        if (lane == 0) {
+          if (half == 0) MFA_TR(kind, ntr[kind]);
           uint8_t* dst = sRing + slot * kSlotBytes;
           const int t0 = t.tile * kTile;
           if (!kPaged) {
@@ -389,8 +553,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             for (int j = 0; j < nsub; ++j) {
               const int tok = t0 + j * rows;
               if (tok >= t.L) break;
-              const int lp = tok / ps;
-              int phys = __ldg(p.page_table + static_cast<int64_t>(t.b) * p.pt_stride + lp);
+              int phys = __ldg(p.page_table + static_cast<int64_t>(t.b) * p.pt_stride + tok / ps);
               if (phys < 0 || phys >= p.num_pages) {
                 record_error(5 /* MFA_ERR_BAD_INDEX */);
                 phys = 0;
@@ -400,74 +563,82 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                             (2 * half + r) * 64, tok % ps, phys, policy);
             }
           }
-          ++item;
         }
-        return true;
-      };
-      TileInfo kt, vt;
-      bool more_k = ks.next(kt);
-      bool first = true;
-      while (ok) {
-        if (more_k) ok = load(kt, &tm_k);
-        if (ok && !first) {
-          vs.next(vt);
-          ok = load(vt, &tm_v);
-        }
-        if (!more_k) break;
-        first = false;
-        more_k = ks.next(kt);
+        __syncwarp();
+        ++item;
       }
-      (void)ok;
+      ++ntr[kind];
+      return true;
+    };
+    TileInfo kt, vt;
+    bool more_k = ks.next(kt);
+    bool first = true, ok = true;
+    while (ok) {
+      if (more_k) ok = load(kt, &tm_k);
+      if (ok && !first) {
+        vs.next(vt);
+        ok = load(vt, &tm_v);
+      }
+      if (!more_k) break;
+      first = false;
+      more_k = ks.next(kt);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =====================================
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_f16(128, 64, 1, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_f16(128, 64, 1, 1, 1);
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t ring_base = smem_u32(sRing);
-      const uint32_t p_base = smem_u32(sP);
-      TileStream qs;
-      qs.init(p, c.b_start, c.off_start, c.tiles);
-      uint32_t item = 0, nq = 0;
-      bool ok = true;
+    constexpr uint32_t idesc_qk = idesc_f16(128, 64, 1, 0, 0);
+    constexpr uint32_t idesc_pv = idesc_f16(128, 64, 1, 1, 1);
+    const uint32_t q_base = smem_u32(sQ);
+    const uint32_t ring_base = smem_u32(sRing);
+    const uint32_t p_base = smem_u32(sP);
+    TileStream qs;
+    qs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    uint32_t item = 0, nq = 0;
+    bool ok = true;
 
-      auto issue_pv = [&](const TileInfo& t, uint32_t j) -> bool {
-        if (!mbar_wait(&c.p_full, par(j), abort_flag)) return false;
-        const uint32_t lo = item++, hi = item++;
-        if (!mbar_wait(&c.slot_full[lo % kSlots], par(lo / kSlots), abort_flag)) return false;
-        if (!mbar_wait(&c.slot_full[hi % kSlots], par(hi / kSlots), abort_flag)) return false;
-        tc_fence_after();
+    auto issue_pv = [&](const TileInfo& t, uint32_t j) -> bool {
+      if (!warp_wait(&c.p_full, par(j), abort_flag)) return false;
+      const uint32_t lo = item++, hi = item++;
+      if (!warp_wait(&c.slot_full[lo % kSlots], par(lo / kSlots), abort_flag)) return false;
+      if (!warp_wait(&c.slot_full[hi % kSlots], par(hi / kSlots), abort_flag)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        MFA_TR(3, j);
         const uint32_t v_lo = ring_base + (lo % kSlots) * kSlotBytes;
         const uint32_t v_hi = ring_base + (hi % kSlots) * kSlotBytes;
+        // head dims 0-127 first, so their ring slot is released half-way
 #pragma unroll
-        for (int s = 0; s < kTile / 16; ++s) {
-          const uint64_t bdesc = sw128_desc(p_base + s * 2048, 8192, 1024);
-          const uint32_t acc = (t.seg_first && s == 0) ? 0u : 1u;
-          mma_f16_ss(tmem + kColOlo, sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024), bdesc,
-                     idesc_pv, acc);
-          mma_f16_ss(tmem + kColOhi, sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024), bdesc,
-                     idesc_pv, acc);
-        }
+        for (int s = 0; s < kTile / 16; ++s)
+          mma_f16_ss(tmem + kColOlo, sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
+                     sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                     (t.seg_first && s == 0) ? 0u : 1u);
         mma_commit(&c.slot_empty[lo % kSlots]);
+#pragma unroll
+        for (int s = 0; s < kTile / 16; ++s)
+          mma_f16_ss(tmem + kColOhi, sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
+                     sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                     (t.seg_first && s == 0) ? 0u : 1u);
         mma_commit(&c.slot_empty[hi % kSlots]);
         mma_commit(&c.o_full);
-        return true;
-      };
+      }
+      __syncwarp();
+      return true;
+    };
 
-      TileInfo cur, prev;
-      uint32_t g = 0;
-      while (ok && qs.next(cur)) {
-        if (cur.seg_first) {
-          ok = mbar_wait(&c.q_full, par(nq), abort_flag);
-          ++nq;
-          if (!ok) break;
-        }
-        if (g >= 2 && !(ok = mbar_wait(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag))) break;
-        const uint32_t lo = item++, hi = item++;
-        if (!(ok = mbar_wait(&c.slot_full[lo % kSlots], par(lo / kSlots), abort_flag))) break;
-        if (!(ok = mbar_wait(&c.slot_full[hi % kSlots], par(hi / kSlots), abort_flag))) break;
-        tc_fence_after();
+    TileInfo cur, prev;
+    uint32_t g = 0;
+    while (ok && qs.next(cur)) {
+      if (cur.seg_first) {
+        ok = warp_wait(&c.q_full, par(nq), abort_flag);
+        ++nq;
+        if (!ok) break;
+      }
+      if (g >= 2 && !(ok = warp_wait(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag))) break;
+      const uint32_t lo = item++, hi = item++;
+      if (!(ok = warp_wait(&c.slot_full[lo % kSlots], par(lo / kSlots), abort_flag))) break;
+      if (!(ok = warp_wait(&c.slot_full[hi % kSlots], par(hi / kSlots), abort_flag))) break;
+      tc_fence_after();
+      if (lane == 0) {
+        MFA_TR(2, g);
         const uint32_t k_lo = ring_base + (lo % kSlots) * kSlotBytes;
         const uint32_t k_hi = ring_base + (hi % kSlots) * kSlotBytes;
         const uint32_t d_s = tmem + kColS + (g & 1) * 64;
@@ -483,72 +654,77 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         mma_commit(&c.slot_empty[hi % kSlots]);
         mma_commit(&c.s_full[g & 1]);
         if (cur.seg_last) mma_commit(&c.q_empty);
-        if (g >= 1 && !(ok = issue_pv(prev, g - 1))) break;
-        prev = cur;
-        ++g;
       }
-      if (ok && g >= 1) ok = issue_pv(prev, g - 1);
-      if (!ok) {
-        // drain: wait (bounded, ignoring the abort flag) for issued MMAs
-        mma_commit(&c.drain);
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(&c.drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+      __syncwarp();
+      if (g >= 1 && !(ok = issue_pv(prev, g - 1))) break;
+      prev = cur;
+      ++g;
+    }
+    if (ok && g >= 1) ok = issue_pv(prev, g - 1);
+    if (!ok && lane == 0) {
+      // drain: wait (bounded, ignoring the abort flag) for issued MMAs
+      mma_commit(&c.drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(&c.drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
       }
     }
+    __syncwarp();
   } else if (warp == 2) {
     // ======================= q producer =====================================
-    if (lane == 0) {
-      const uint64_t policy = l2_policy_evict_last();
-      TileStream qs;
-      qs.init(p, c.b_start, c.off_start, c.tiles);
-      TileInfo t;
-      uint32_t k = 0;
-      while (qs.next(t)) {
-        if (!t.seg_first) continue;
-        if (!mbar_wait(&c.q_empty, par(k) ^ 1u, abort_flag)) break;
+    const uint64_t policy = l2_policy_evict_last();
+    TileStream qs, ahead;
+    qs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    ahead.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    TileInfo t, ta;
+    bool more_ahead = ahead.next(ta);  // stays one segment ahead of qs
+    uint32_t k = 0;
+    while (qs.next(t)) {
+      if (!t.seg_first) continue;
+      if (!warp_wait(&c.q_empty, par(k) ^ 1u, abort_flag)) break;
+      if (lane == 0) {
         mbar_arrive_expect_tx(&c.q_full, kQBytes);
         for (int r = 0; r < 4; ++r)
           tma_load_3d(sQ + r * 8192, &tm_q, &c.q_full, r * 64, 0, t.b, policy);
-        ++k;
       }
+      // pull the next segment's q rows into L2 while this segment runs
+      while (more_ahead && (ta.b == t.b || !ta.seg_first)) more_ahead = ahead.next(ta);
+      if (more_ahead && lane == 0)
+        for (int r = 0; r < 4; ++r) tma_prefetch_3d(&tm_q, r * 64, 0, ta.b);
+      __syncwarp();
+      ++k;
     }
   } else if (warp >= 4) {
     // ======================= softmax + epilogue =============================
-    const int sub = warp & 3;                 // TMEM sub-partition of this warp
-    const int row = sub * 32 + lane;          // token row in S^T / dim row in O^T
+    const int wg = (warp - 4) >> 2;   // heads [32 wg, 32 wg + 32)
+    const int sub = warp & 3;         // TMEM sub-partition of this warp
+    const int row = sub * 32 + lane;  // token row in S^T / head-dim row in O^T
+    const int hbase = wg * kWGHeads;
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
     TileStream ts;
-    ts.init(p, c.b_start, c.off_start, c.tiles);
+    ts.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
     TileInfo t;
     uint32_t g = 0, nseg = 0;
-    float m_run0 = -INFINITY, m_run1 = -INFINITY;  // running max, heads 2*lane, 2*lane+1
-    float l_part[kHeads];
+    float m_run = -INFINITY;  // running max in use (log2 units), head hbase + lane
+    float l_part[kWGHeads];
 #pragma unroll
-    for (int h = 0; h < kHeads; ++h) l_part[h] = 0.f;
+    for (int h = 0; h < kWGHeads; ++h) l_part[h] = 0.f;
     const float sl2 = p.score_log2;
+    float* mv = c.mv[wg][sub];
+    float* cv = c.cv[wg][sub];
 
     while (ts.next(t)) {
-      if (t.seg_first) {
-        m_run0 = m_run1 = -INFINITY;
-#pragma unroll
-        for (int h = 0; h < kHeads; ++h) l_part[h] = 0.f;
-      }
-      // ---- scores of this tile ----------------------------------------
-      if (!mbar_wait(&c.s_full[g & 1], par(g >> 1), abort_flag)) break;
+      if (t.seg_first) m_run = -INFINITY;  // (l_part is zero at every segment start)
+      // ---- scores of this tile (this warpgroup's 32 heads) ---------------
+      if (!warp_wait(&c.s_full[g & 1], par(g >> 1), abort_flag)) break;
+      if (warp == 4 && lane == 0) MFA_TR(4, g);
       tc_fence_after();
-      float s[kHeads];
+      float s[kWGHeads];
       {
         uint32_t r[32];
-        const uint32_t a = tmem + lane_addr + kColS + (g & 1) * 64;
-        tmem_ld32(a, r);
+        tmem_ld32(tmem + lane_addr + kColS + (g & 1) * 64 + hbase, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 32; ++h) s[h] = __uint_as_float(r[h]);
-        tmem_ld32(a + 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) s[32 + h] = __uint_as_float(r[h]);
+        for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]);
       }
       tc_fence_before();
       __syncwarp();
@@ -557,365 +733,322 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int valid = min(kTile, t.L - t.tile * kTile);
       const bool row_ok = row < valid;
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) s[h] = row_ok ? s[h] * sl2 : -INFINITY;
+      for (int h = 0; h < kWGHeads; ++h) s[h] = row_ok ? s[h] * sl2 : -INFINITY;
 
       // ---- per-head maximum over the tile's 128 rows --------------------
       {
-        float v[kHeads];
+        float v[kWGHeads];
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) v[h] = s[h];
-        reduce_scatter64<true>(v, lane);
-        c.red[g & 1][sub][2 * lane] = v[0];
-        c.red[g & 1][sub][2 * lane + 1] = v[1];
+        for (int h = 0; h < kWGHeads; ++h) v[h] = s[h];
+        c.red[g & 1][wg][sub][lane] = reduce_scatter32<true>(v, lane);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&c.red_full[g & 1]);
-      if (!mbar_wait(&c.red_full[g & 1], par(g >> 1), abort_flag)) break;
-      float tmax0 = c.red[g & 1][0][2 * lane], tmax1 = c.red[g & 1][0][2 * lane + 1];
-#pragma unroll
-      for (int w = 1; w < 4; ++w) {
-        tmax0 = fmaxf(tmax0, c.red[g & 1][w][2 * lane]);
-        tmax1 = fmaxf(tmax1, c.red[g & 1][w][2 * lane + 1]);
-      }
+      if (lane == 0) mbar_arrive(&c.red_full[wg][g & 1]);
+      if (!warp_wait(&c.red_full[wg][g & 1], par(g >> 1), abort_flag)) break;
+      if (warp == 4 && lane == 0) MFA_TR(5, g);
+      const float tmax = fmaxf(fmaxf(c.red[g & 1][wg][0][lane], c.red[g & 1][wg][1][lane]),
+                               fmaxf(c.red[g & 1][wg][2][lane], c.red[g & 1][wg][3][lane]));
       // lazy rescaling: move the reference max only when the tile's max
       // exceeds it by more than the threshold (exact: the factor cancels)
-      float m_new0 = m_run0, m_new1 = m_run1, corr0 = 1.f, corr1 = 1.f;
-      if (tmax0 > m_run0 + kRescaleThreshold) {
-        m_new0 = tmax0;
-        corr0 = ex2_approx(m_run0 - tmax0);
+      float corr = 1.f;
+      if (tmax > m_run + kRescaleThreshold) {
+        corr = ex2_approx(m_run - tmax);
+        m_run = tmax;
       }
-      if (tmax1 > m_run1 + kRescaleThreshold) {
-        m_new1 = tmax1;
-        corr1 = ex2_approx(m_run1 - tmax1);
-      }
-      m_run0 = m_new0;
-      m_run1 = m_new1;
-      const bool rescale = __any_sync(0xffffffffu, corr0 != 1.f || corr1 != 1.f);
-      c.mv[sub][2 * lane] = m_new0;
-      c.mv[sub][2 * lane + 1] = m_new1;
-      c.cv[sub][2 * lane] = corr0;
-      c.cv[sub][2 * lane + 1] = corr1;
+      const bool rescale = __any_sync(0xffffffffu, corr != 1.f);
+      mv[lane] = m_run;
+      cv[lane] = corr;
       __syncwarp();
 
       // ---- probabilities, row sums ---------------------------------------
-      uint32_t pk[kHeads / 2];
+      uint32_t pk[kWGHeads / 2];
 #pragma unroll
-      for (int h = 0; h < kHeads; h += 2) {
-        const float2 m2 = *reinterpret_cast<const float2*>(&c.mv[sub][h]);
-        const float p0 = ex2_approx(s[h] - m2.x);
-        const float p1 = ex2_approx(s[h + 1] - m2.y);
+      for (int h = 0; h < kWGHeads; h += 4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(&mv[h]);
+        const float p0 = ex2_approx(s[h] - m4.x);
+        const float p1 = ex2_approx(s[h + 1] - m4.y);
+        const float p2 = ex2_approx(s[h + 2] - m4.z);
+        const float p3 = ex2_approx(s[h + 3] - m4.w);
         if (rescale) {
-          const float2 c2 = *reinterpret_cast<const float2*>(&c.cv[sub][h]);
-          l_part[h] = l_part[h] * c2.x + p0;
-          l_part[h + 1] = l_part[h + 1] * c2.y + p1;
+          const float4 c4 = *reinterpret_cast<const float4*>(&cv[h]);
+          l_part[h] = l_part[h] * c4.x + p0;
+          l_part[h + 1] = l_part[h + 1] * c4.y + p1;
+          l_part[h + 2] = l_part[h + 2] * c4.z + p2;
+          l_part[h + 3] = l_part[h + 3] * c4.w + p3;
         } else {
           l_part[h] += p0;
           l_part[h + 1] += p1;
+          l_part[h + 2] += p2;
+          l_part[h + 3] += p3;
         }
         pk[h / 2] = pack_bf16x2(p0, p1);
+        pk[h / 2 + 1] = pack_bf16x2(p2, p3);
       }
 
       // ---- P buffer and O are free once the previous tile's PV completed --
-      if (g >= 1 && !mbar_wait(&c.o_full, par(g - 1), abort_flag)) break;
+      if (warp == 4 && lane == 0) MFA_TR(6, g);
+      if (g >= 1 && !warp_wait(&c.o_full, par(g - 1), abort_flag)) break;
       tc_fence_after();
       if (rescale && !t.seg_first) {
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {  // (O_lo, O_hi) x two 16-column chunks
+          uint32_t r[16];
+          const int cb = (q4 & 1) * 16;
+          const uint32_t a = tmem + lane_addr + ((q4 >> 1) ? kColOhi : kColOlo) + hbase + cb;
+          tmem_ld16(a, r);
+          tmem_wait_ld();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-          for (int cb = 0; cb < 2; ++cb) {
-            uint32_t r[32];
-            const uint32_t a = tmem + lane_addr + (half ? kColOhi : kColOlo) + cb * 32;
-            tmem_ld32(a, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              r[j] = __float_as_uint(__uint_as_float(r[j]) * c.cv[sub][cb * 32 + j]);
-            tmem_st32(a, r);
-          }
+          for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * cv[cb + j]);
+          tmem_st16(a, r);
         }
         tmem_wait_st();
       }
       {
         const uint32_t rowaddr = smem_u32(sP) + row * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(rowaddr + ((ch ^ (row & 7)) << 4), pk[4 * ch], pk[4 * ch + 1],
+        for (int ch = 0; ch < 4; ++ch)
+          st_shared_v4(rowaddr + (((4 * wg + ch) ^ (row & 7)) << 4), pk[4 * ch], pk[4 * ch + 1],
                        pk[4 * ch + 2], pk[4 * ch + 3]);
       }
       // rows past the sequence end: zero the V rows so 0 * (stale or NaN) never
-      // reaches the accumulator
+      // reaches the accumulator (warpgroup 0: head dims 0-127, 1: 128-255)
       if (valid < kTile) {
-        const uint32_t it = v_item(g, t.cta_last);
-        bool ok = mbar_wait(&c.slot_full[it % kSlots], par(it / kSlots), abort_flag);
-        ok = ok && mbar_wait(&c.slot_full[(it + 1) % kSlots], par((it + 1) / kSlots), abort_flag);
-        if (!ok) break;
+        const uint32_t it = v_item(g, t.cta_last) + wg;
+        if (!warp_wait(&c.slot_full[it % kSlots], par(it / kSlots), abort_flag)) break;
         if (!row_ok) {
+          const uint32_t base = smem_u32(sRing) + (it % kSlots) * kSlotBytes + row * 128;
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t base = smem_u32(sRing) + ((it + hh) % kSlots) * kSlotBytes + row * 128;
+          for (int r = 0; r < 2; ++r)
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch)
-                st_shared_v4(base + r * (kSlotBytes / 2) + ch * 16, 0u, 0u, 0u, 0u);
-          }
+            for (int ch = 0; ch < 8; ++ch)
+              st_shared_v4(base + r * (kSlotBytes / 2) + ch * 16, 0u, 0u, 0u, 0u);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.p_full);
+      if (warp == 4 && lane == 0) MFA_TR(7, g);
 
       // ---- epilogue at the end of a segment -------------------------------
       if (t.seg_last) {
-        // row sums: reduce the 128 rows' partial sums per head
         {
-          float v[kHeads];
+          float v[kWGHeads];
 #pragma unroll
-          for (int h = 0; h < kHeads; ++h) v[h] = l_part[h];
-          reduce_scatter64<false>(v, lane);
-          c.lred[sub][2 * lane] = v[0];
-          c.lred[sub][2 * lane + 1] = v[1];
+          for (int h = 0; h < kWGHeads; ++h) v[h] = l_part[h];
+          c.lred[wg][sub][lane] = reduce_scatter32<false>(v, lane);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&c.l_full);
-        if (!mbar_wait(&c.l_full, par(nseg), abort_flag)) break;
-        const float l0 = c.lred[0][2 * lane] + c.lred[1][2 * lane] + c.lred[2][2 * lane] +
-                         c.lred[3][2 * lane];
-        const float l1 = c.lred[0][2 * lane + 1] + c.lred[1][2 * lane + 1] +
-                         c.lred[2][2 * lane + 1] + c.lred[3][2 * lane + 1];
-        // this warp's copy: 1/l in cv, lse (natural log) in mv
-        __syncwarp();
-        c.cv[sub][2 * lane] = p.out_scale / l0;
-        c.cv[sub][2 * lane + 1] = p.out_scale / l1;
-        const float lse0 = (m_run0 + lg2_approx(l0)) * kLn2;
-        const float lse1 = (m_run1 + lg2_approx(l1)) * kLn2;
-        c.mv[sub][2 * lane] = lse0;
-        c.mv[sub][2 * lane + 1] = lse1;
+        if (lane == 0) mbar_arrive(&c.l_full[wg]);
+        if (!warp_wait(&c.l_full[wg], par(nseg), abort_flag)) break;
+        const float l = c.lred[wg][0][lane] + c.lred[wg][1][lane] + c.lred[wg][2][lane] +
+                        c.lred[wg][3][lane];
+        // the next tile starts a new segment: the row sums restart from zero
+#pragma unroll
+        for (int h = 0; h < kWGHeads; ++h) l_part[h] = 0.f;
+        const float lse = (m_run + lg2_approx(l)) * kLn2;  // head hbase + lane
+        cv[lane] = p.out_scale / l;
         if (sub == 0) {
-          if (t.slot >= 0) {
-            p.ws_lse[static_cast<int64_t>(t.slot) * kHeads + 2 * lane] = lse0;
-            p.ws_lse[static_cast<int64_t>(t.slot) * kHeads + 2 * lane + 1] = lse1;
-          } else if (p.lse_out) {
-            p.lse_out[t.b * p.lse_sb + 2 * lane] = lse0;
-            p.lse_out[t.b * p.lse_sb + 2 * lane + 1] = lse1;
-          }
+          if (t.slot >= 0)
+            p.ws_lse[static_cast<int64_t>(t.slot) * kHeads + hbase + lane] = lse;
+          else if (p.lse_out)
+            p.lse_out[t.b * p.lse_sb + hbase + lane] = lse;
         }
         __syncwarp();
-        // O = O^T / l, written row (head-dim index) by row
-        if (!mbar_wait(&c.o_full, par(g), abort_flag)) break;
+        if (!warp_wait(&c.o_full, par(g), abort_flag)) break;
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           const int d = half * 128 + row;
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_addr + (half ? kColOhi : kColOlo) + hbase, r);
+          tmem_wait_ld();
+          if (t.slot >= 0) {
+            // partial layout [slot][head][d]: a warp writes 128 contiguous bytes per head
+            float* dst = p.ws_o + static_cast<int64_t>(t.slot) * kPartialFloats +
+                         static_cast<int64_t>(hbase) * kDim + d;
 #pragma unroll
-          for (int cb = 0; cb < 2; ++cb) {
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_addr + (half ? kColOhi : kColOlo) + cb * 32, r);
-            tmem_wait_ld();
-            if (t.slot >= 0) {
-              float* dst = p.ws_o + static_cast<int64_t>(t.slot) * kPartialFloats + d;
+            for (int j = 0; j < 32; ++j) dst[j * kDim] = __uint_as_float(r[j]) * cv[j];
+          } else {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int h = cb * 32 + j;
-                dst[h * kDim] = __uint_as_float(r[j]) * c.cv[sub][h];
-              }
-            } else if (p.out_f32) {
-              float* dst = static_cast<float*>(p.out) + t.b * p.out_sb + d;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int h = cb * 32 + j;
-                dst[h * p.out_sh] = __uint_as_float(r[j]) * c.cv[sub][h];
-              }
-            } else {
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + t.b * p.out_sb + d;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int h = cb * 32 + j;
-                dst[h * p.out_sh] = __float2bfloat16_rn(__uint_as_float(r[j]) * c.cv[sub][h]);
-              }
-            }
+            for (int j = 0; j < 32; ++j)
+              store_out(p, t.b, hbase + j, d, __uint_as_float(r[j]) * cv[j]);
           }
         }
         tc_fence_before();
+        if (warp == 4 && lane == 0) MFA_TR(8, g);
         ++nseg;
+
       }
       ++g;
     }
   }
 
   // ---- teardown ------------------------------------------------------------
+  if (tid == 0) MFA_TR(11, 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-}
-
-// ===========================================================================
-// Split merge: one CTA per sequence, thread = head-dim index.
-// ===========================================================================
-// Balanced plan: slot of the i-th CTA (counting from c_first) that holds part of
-// a split sequence, or -1 when that CTA's tile range is empty (more CTAs than
-// tiles).
-__device__ __forceinline__ int balanced_slot(int i, int c_first, int slot_of_first,
-                                             long long N, long long G) {
-  if (i == 0) return slot_of_first;
-  const long long cc = c_first + i;
-  const long long lo = (cc * N) / G, hi = ((cc + 1) * N) / G;
-  return hi > lo ? static_cast<int>(2 * cc) : -1;
-}
-
-__global__ void __launch_bounds__(256) mfa_combine_kernel(const DecodeParams p) {
-  const int b = blockIdx.x;
-  const int d = threadIdx.x;
-  __shared__ float s_lse[64][kHeads + 1];  // per slot (chunked) x head
-  __shared__ int s_slot[64];
-  __shared__ float s_m[kHeads], s_wsum[kHeads];
-
-  int L = __ldg(p.seq_lens + b);
-  if (L < 0 || L > p.cap_tokens) L = 0;  // recorded by the attention kernel
-  const int nt = (L + kTile - 1) / kTile;
-
-  // the list of partial slots of this sequence, in plan order
-  int nslots = 0;
-  int slot_of_first = 0, c_first = 0, c_last = -1;
-  long long nt_total = 0;
-  if (nt > 0) {
-    if (p.num_splits == 0) {
-      const long long S = __ldg(p.ws_prefix + b);
-      const long long N = __ldg(p.ws_prefix + p.batch);
-      const long long G = p.grid;
-      nt_total = N;
-      auto owner = [&](long long tt) -> int {
-        return static_cast<int>(((tt + 1) * G - 1) / N);
-      };
-      c_first = owner(S);
-      c_last = owner(S + nt - 1);
-      if (c_first == c_last) return;  // written directly by the attention kernel
-      const long long start_first = (static_cast<long long>(c_first) * N) / G;
-      slot_of_first = (start_first < S) ? 2 * c_first + 1 : 2 * c_first;
-      nslots = c_last - c_first + 1;
-    } else {
-      const int s = p.num_splits;
-      int nonempty = 0;
-      for (int j = 0; j < s; ++j) {
-        const int lo = static_cast<int>((static_cast<long long>(j) * nt) / s);
-        const int hi = static_cast<int>((static_cast<long long>(j + 1) * nt) / s);
-        nonempty += hi > lo;
-      }
-      if (nonempty <= 1) return;
-      nslots = s;  // empty units are skipped below
-    }
+#ifdef MFA_TRACE
+  if (tid == 0) {
+    MFA_GT(0, blockIdx.x, 2, gt_call);
+    if (blockIdx.x < kGtCtas) g_mfa_cnt[blockIdx.x] = gt_call + 1;
   }
+#endif
+}
 
-  if (nt == 0) {
-    // empty sequence: zeros, lse = -inf
-    for (int h = 0; h < kHeads; ++h) {
-      if (p.out_f32)
-        static_cast<float*>(p.out)[b * p.out_sb + h * p.out_sh + d] = 0.f;
-      else
-        static_cast<__nv_bfloat16*>(p.out)[b * p.out_sb + h * p.out_sh + d] =
-            __float2bfloat16_rn(0.f);
+// ===========================================================================
+// Split merge (Flash-Decoding's log-sum-exp combine) and empty sequences.
+// CTA (b, q): sequence b, heads 16q..16q+15; thread = head-dim index.
+//   lse* = max_s lse_s,  w_s = exp(lse_s - lse*),
+//   out = sum_s w_s O_s / sum_s w_s,   lse = lse* + log(sum_s w_s)
+// over the sequence's partials in plan order.
+// ===========================================================================
+constexpr int kCombineHeads = 32;  // heads per CTA
+constexpr int kCombineChunk = 64;  // partial slots staged in shared memory at a time
+
+__global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams p) {
+#ifdef MFA_TRACE
+  const unsigned long long gt_start = global_timer_ns();
+  const int cta_lin = blockIdx.x * gridDim.y + blockIdx.y;
+#endif
+  griddep_wait();  // partials, prefix and lengths come from the attention kernel
+  griddep_launch_dependents();
+#ifdef MFA_TRACE
+  const int gt_call = cta_lin < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[kGtCtas + cta_lin]) : -1;
+  if (threadIdx.x == 0) {
+    MFA_GT(1, cta_lin, 1, gt_call);
+    if (gt_call >= 0 && gt_call < kGtCalls && cta_lin < kGtCtas)
+      g_mfa_gt[((gt_call * 2 + 1) * kGtCtas + cta_lin) * 3] = gt_start;
+  }
+  struct GtEnd {
+    int call, cta;
+    __device__ ~GtEnd() {
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        MFA_GT(1, cta, 2, call);
+        if (cta < kGtCtas) g_mfa_cnt[kGtCtas + cta] = call + 1;
+      }
     }
-    if (p.lse_out && d < kHeads) p.lse_out[b * p.lse_sb + d] = -INFINITY;
+  } gt_end{gt_call, cta_lin};
+#endif
+  __shared__ int s_slot[kCombineChunk];
+  __shared__ float s_w[kCombineChunk][kCombineHeads];  // lse, then weights
+  __shared__ float s_m[kCombineHeads], s_l[kCombineHeads], s_scale[kCombineHeads];
+  const int b = blockIdx.x;
+  const int h0 = blockIdx.y * kCombineHeads;
+  const int d = threadIdx.x;
+
+  const int L = valid_len(p, b);
+  const int nt = tiles_of(L);
+  if (nt == 0) {
+#pragma unroll
+    for (int j = 0; j < kCombineHeads; ++j) store_out(p, b, h0 + j, d, 0.f);
+    if (p.lse_out && d < kCombineHeads) p.lse_out[b * p.lse_sb + h0 + d] = -INFINITY;
     return;
   }
+  SplitList sl;
+  if (p.num_splits == 0)
+    sl.init_balanced(__ldg(p.ws_prefix + b), nt, __ldg(p.ws_prefix + p.batch), p.grid);
+  else
+    sl.init_fixed(b, nt, p.num_splits);
+  if (sl.nonempty() <= 1) return;  // written directly by the attention kernel
 
-  // pass over slots in chunks of 64 to find the per-head max and weight sum
-  float acc[kHeads];
-#pragma unroll
-  for (int h = 0; h < kHeads; ++h) acc[h] = 0.f;
-  if (d < kHeads) {
+  if (d < kCombineHeads) {
     s_m[d] = -INFINITY;
-    s_wsum[d] = 0.f;
+    s_l[d] = 0.f;
+  }
+  float acc[kCombineHeads];
+#pragma unroll
+  for (int j = 0; j < kCombineHeads; ++j) acc[j] = 0.f;
+  for (int base = 0; base < sl.count; base += kCombineChunk) {
+    const int cnt = min(kCombineChunk, sl.count - base);
+    __syncthreads();
+    if (d < cnt) s_slot[d] = sl.slot(base + d);
+    __syncthreads();
+    for (int e = d; e < cnt * kCombineHeads; e += kDim) {
+      const int i = e / kCombineHeads, h = e % kCombineHeads;
+      const int sidx = s_slot[i];
+      s_w[i][h] = sidx >= 0 ? __ldcg(p.ws_lse + static_cast<int64_t>(sidx) * kHeads + h0 + h) : -INFINITY;
+    }
+    __syncthreads();
+    // running max / sum per head over the chunk (online across chunks); rescale acc
+    float scale_old = 1.f;
+    if (d < kCombineHeads) {
+      const float m_old = s_m[d];
+      float m = m_old;
+      for (int i = 0; i < cnt; ++i) m = fmaxf(m, s_w[i][d]);
+      float l = s_l[d] * ex2_approx((m_old - m) * kLog2e);
+      for (int i = 0; i < cnt; ++i) {
+        const float w = ex2_approx((s_w[i][d] - m) * kLog2e);
+        s_w[i][d] = w;
+        l += w;
+      }
+      s_m[d] = m;
+      s_l[d] = l;
+      scale_old = ex2_approx((m_old - m) * kLog2e);
+    }
+    if (d < kCombineHeads) s_scale[d] = scale_old;
+    __syncthreads();
+    if (base > 0) {
+#pragma unroll
+      for (int j = 0; j < kCombineHeads; ++j) acc[j] *= s_scale[j];
+    }
+    int i = 0;
+    for (; i + 1 < cnt; i += 2) {  // two slots' loads in flight together
+      const int sa = s_slot[i], sb = s_slot[i + 1];
+      // partial layout [slot][head][d]: thread d, consecutive threads read consecutive d
+      const float* pa = p.ws_o + static_cast<int64_t>(sa < 0 ? 0 : sa) * kPartialFloats +
+                        static_cast<int64_t>(h0) * kDim + d;
+      const float* pb = p.ws_o + static_cast<int64_t>(sb < 0 ? 0 : sb) * kPartialFloats +
+                        static_cast<int64_t>(h0) * kDim + d;
+      float va[kCombineHeads], vb[kCombineHeads];
+#pragma unroll
+      for (int j = 0; j < kCombineHeads; ++j) {
+        va[j] = sa >= 0 ? __ldcg(pa + j * kDim) : 0.f;
+        vb[j] = sb >= 0 ? __ldcg(pb + j * kDim) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < kCombineHeads; ++j) acc[j] += s_w[i][j] * va[j] + s_w[i + 1][j] * vb[j];
+    }
+    if (i < cnt) {
+      const int sa = s_slot[i];
+      if (sa >= 0) {
+        const float* pa = p.ws_o + static_cast<int64_t>(sa) * kPartialFloats +
+                          static_cast<int64_t>(h0) * kDim + d;
+#pragma unroll
+        for (int j = 0; j < kCombineHeads; ++j) acc[j] += s_w[i][j] * __ldcg(pa + j * kDim);
+      }
+    }
   }
   __syncthreads();
-  // first pass: maxima
-  for (int base = 0; base < nslots; base += 64) {
-    const int cnt = min(64, nslots - base);
-    if (d < cnt) {
-      int slot;
-      const int i = base + d;
-      if (p.num_splits == 0) {
-        slot = balanced_slot(i, c_first, slot_of_first, nt_total, p.grid);
-      } else {
-        const int s = p.num_splits;
-        const int lo = static_cast<int>((static_cast<long long>(i) * nt) / s);
-        const int hi = static_cast<int>((static_cast<long long>(i + 1) * nt) / s);
-        slot = (hi > lo) ? b * s + i : -1;
-      }
-      s_slot[d] = slot;
-    }
-    __syncthreads();
-    for (int e = d; e < cnt * kHeads; e += blockDim.x) {
-      const int i = e / kHeads, h = e % kHeads;
-      const int slot = s_slot[i];
-      s_lse[i][h] = slot >= 0 ? __ldg(p.ws_lse + static_cast<int64_t>(slot) * kHeads + h)
-                              : -INFINITY;
-    }
-    __syncthreads();
-    if (d < kHeads) {
-      float m = s_m[d];
-      for (int i = 0; i < cnt; ++i) m = fmaxf(m, s_lse[i][d]);
-      s_m[d] = m;
-    }
-    __syncthreads();
-  }
-  // second pass: weighted sums
-  for (int base = 0; base < nslots; base += 64) {
-    const int cnt = min(64, nslots - base);
-    if (d < cnt) {
-      int slot;
-      const int i = base + d;
-      if (p.num_splits == 0) {
-        slot = balanced_slot(i, c_first, slot_of_first, nt_total, p.grid);
-      } else {
-        const int s = p.num_splits;
-        const int lo = static_cast<int>((static_cast<long long>(i) * nt) / s);
-        const int hi = static_cast<int>((static_cast<long long>(i + 1) * nt) / s);
-        slot = (hi > lo) ? b * s + i : -1;
-      }
-      s_slot[d] = slot;
-    }
-    __syncthreads();
-    for (int e = d; e < cnt * kHeads; e += blockDim.x) {
-      const int i = e / kHeads, h = e % kHeads;
-      const int slot = s_slot[i];
-      const float l = slot >= 0 ? __ldg(p.ws_lse + static_cast<int64_t>(slot) * kHeads + h)
-                                : -INFINITY;
-      s_lse[i][h] = (slot >= 0) ? expf(l - s_m[h]) : 0.f;
-    }
-    __syncthreads();
-    if (d < kHeads) {
-      float w = s_wsum[d];
-      for (int i = 0; i < cnt; ++i) w += s_lse[i][d];
-      s_wsum[d] = w;
-    }
-    for (int i = 0; i < cnt; ++i) {
-      const int slot = s_slot[i];
-      if (slot < 0) continue;
-      const float* src = p.ws_o + static_cast<int64_t>(slot) * kPartialFloats + d;
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) acc[h] += s_lse[i][h] * __ldg(src + h * kDim);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int h = 0; h < kHeads; ++h) {
-    const float o = acc[h] / s_wsum[h];
-    if (p.out_f32)
-      static_cast<float*>(p.out)[b * p.out_sb + h * p.out_sh + d] = o;
-    else
-      static_cast<__nv_bfloat16*>(p.out)[b * p.out_sb + h * p.out_sh + d] =
-          __float2bfloat16_rn(o);
-  }
-  if (p.lse_out && d < kHeads) p.lse_out[b * p.lse_sb + d] = s_m[d] + logf(s_wsum[d]);
+  for (int j = 0; j < kCombineHeads; ++j) store_out(p, b, h0 + j, d, acc[j] / s_l[j]);
+  if (p.lse_out && d < kCombineHeads)
+    p.lse_out[b * p.lse_sb + h0 + d] = s_m[d] + lg2_approx(s_l[d]) * kLn2;
 }
 
 // ===========================================================================
-// host-side launch helpers (called from mfa_api.cu)
+// host-side launch helper (called from mfa_api.cu)
 // ===========================================================================
 int decode_smem_bytes() { return kSmemBytes; }
+
+template <typename Kernel, typename... Args>
+static cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 cudaError_t launch_decode(bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
                           const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
@@ -931,14 +1064,13 @@ cudaError_t launch_decode(bool paged, const CUtensorMap& tq, const CUtensorMap& 
     if (err != cudaSuccess) return err;
     configured_dev[paged ? 1 : 0] = dev;
   }
-  if (paged)
-    mfa_decode_kernel<true><<<p.grid, kDecodeThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
-  else
-    mfa_decode_kernel<false><<<p.grid, kDecodeThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
-  err = cudaGetLastError();
+  err = paged ? launch_pdl(mfa_decode_kernel<true>, dim3(p.grid), dim3(kDecodeThreads),
+                           kSmemBytes, stream, tq, tk, tv, p)
+              : launch_pdl(mfa_decode_kernel<false>, dim3(p.grid), dim3(kDecodeThreads),
+                           kSmemBytes, stream, tq, tk, tv, p);
   if (err != cudaSuccess) return err;
-  mfa_combine_kernel<<<p.batch, 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(mfa_combine_kernel, dim3(p.batch, kHeads / kCombineHeads), dim3(kDim), 0,
+                    stream, p);
 }
 
 }  // namespace mfa

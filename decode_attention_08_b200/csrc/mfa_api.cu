@@ -23,6 +23,14 @@ using namespace mfa;
 
 namespace {
 
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+// Records a failed CUDA call for mfa_last_cuda_error_string(); returns MFA_ERR_CUDA.
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = e;
+  return MFA_ERR_CUDA;
+}
+
 constexpr int kMaxDevices = 64;
 
 // ---------------------------------------------------------------------------
@@ -151,18 +159,20 @@ int cached_workspace(CachedWs* table, size_t need, bool zero, void** out) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Decode workspace: the plan's per-sequence tile prefix, then the partial
+// outputs of split sequences and their log-sum-exp values.
 struct DecodeWsLayout {
-  size_t o_off, lse_off, prefix_off, total;
+  size_t prefix_off, o_off, lse_off, total;
   int slots;
 };
 
 DecodeWsLayout decode_ws_layout(int batch, int num_splits, int grid) {
   DecodeWsLayout l;
   l.slots = num_splits == 0 ? 2 * grid : batch * num_splits;
-  l.o_off = 0;
+  l.prefix_off = 0;
+  l.o_off = align256(static_cast<size_t>(batch + 1) * sizeof(int));
   l.lse_off = align256(l.o_off + static_cast<size_t>(l.slots) * kPartialFloats * sizeof(float));
-  l.prefix_off = align256(l.lse_off + static_cast<size_t>(l.slots) * kHeads * sizeof(float));
-  l.total = align256(l.prefix_off + static_cast<size_t>(batch + 1) * sizeof(int));
+  l.total = align256(l.lse_off + static_cast<size_t>(l.slots) * kHeads * sizeof(float));
   return l;
 }
 
@@ -182,6 +192,11 @@ struct QprojWsLayout {
   int splits;
 };
 
+// The split-K counters sit in a fixed region at the start of the workspace so
+// that calls of any shape reuse the same zero-filled counters (every call
+// leaves them zero); partials and the latent follow.
+constexpr int kMaxCounters = 1024;  // output tiles of the first GEMM: rank <= 128 * 1024
+
 QprojWsLayout qproj_ws_layout(int batch, int dm, int rank, int sms) {
   QprojWsLayout l;
   const int k_blocks = dm / 64;
@@ -190,9 +205,9 @@ QprojWsLayout qproj_ws_layout(int batch, int dm, int rank, int sms) {
   if (splits < 1) splits = 1;
   if (splits > k_blocks) splits = k_blocks;
   l.splits = splits;
-  l.part_off = 0;
-  l.cnt_off = align256(static_cast<size_t>(splits) * batch * rank * sizeof(float));
-  l.lat_off = align256(l.cnt_off + static_cast<size_t>(m_tiles) * sizeof(int));
+  l.cnt_off = 0;
+  l.part_off = align256(static_cast<size_t>(kMaxCounters) * sizeof(int));
+  l.lat_off = align256(l.part_off + static_cast<size_t>(splits) * batch * rank * sizeof(float));
   l.total = align256(l.lat_off + static_cast<size_t>(2 * batch) * rank * 2);
   return l;
 }
@@ -218,6 +233,27 @@ const char* mfa_error_string(int code) {
 }
 
 int mfa_version(void) { return 100; }
+
+#ifdef MFA_TRACE
+// Trace builds only: copy the pipeline trace (see decode_kernel.cu) to host memory.
+int mfa_debug_read_trace(void* dst, size_t bytes) {
+  if (bytes > sizeof(g_mfa_trace)) bytes = sizeof(g_mfa_trace);
+  return cudaMemcpyFromSymbol(dst, g_mfa_trace, bytes) == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+}
+int mfa_debug_read_timeline(void* dst, size_t bytes) {
+  if (bytes > sizeof(g_mfa_gt)) bytes = sizeof(g_mfa_gt);
+  return cudaMemcpyFromSymbol(dst, g_mfa_gt, bytes) == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+}
+int mfa_debug_reset_timeline(void) {
+  static int zeros[2 * kGtCtas] = {0};
+  return cudaMemcpyToSymbol(g_mfa_cnt, zeros, sizeof zeros) == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+}
+#endif
+
+const char* mfa_last_cuda_error_string(void) {
+  return t_last_cuda_error == cudaSuccess ? "no CUDA error recorded"
+                                          : cudaGetErrorString(t_last_cuda_error);
+}
 
 size_t mfa_decode_workspace_size(int batch, int num_splits) {
   if (batch <= 0 || num_splits < 0 || num_splits > kMaxSplits) return 0;
@@ -352,7 +388,7 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
   p.ws_prefix = reinterpret_cast<int*>(ws + wl.prefix_off);
 
   const cudaError_t err = launch_decode(paged, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream));
-  return err == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+  return err == cudaSuccess ? MFA_OK : cuda_fail(err);
 }
 
 }  // namespace
@@ -411,7 +447,7 @@ int qproj_impl(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_
   if (w_qa->shape[0] != Dm || w_qb->shape[0] != R || q_out->shape[0] != B || q_out->shape[1] != N)
     return MFA_ERR_INVALID_ARG;
   if (B < 1 || B > 128 || Dm % 64 || R % 128 || N % 128 || Dm <= 0 || R <= 0 || N <= 0 ||
-      Dm > (1 << 20) || R > (1 << 20) || N > (1 << 24))
+      Dm > (1 << 20) || R > 128 * kMaxCounters || N > (1 << 24))
     return MFA_ERR_UNSUPPORTED;
   if (validate_only) return MFA_OK;
 
@@ -446,7 +482,8 @@ int qproj_impl(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_
   p1.counters = reinterpret_cast<int*>(ws + wl.cnt_off);
   p1.latent = latent;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (launch_qproj(tw1, tx, p1, static_cast<int>(R / 128), st) != cudaSuccess) return MFA_ERR_CUDA;
+  cudaError_t e = launch_qproj(tw1, tx, p1, static_cast<int>(R / 128), st);
+  if (e != cudaSuccess) return cuda_fail(e);
 
   QprojParams p2 = p1;
   p2.k_blocks = static_cast<int>(R / 64);
@@ -456,7 +493,8 @@ int qproj_impl(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_
   p2.mode = 1;
   p2.q_out = static_cast<__nv_bfloat16*>(q_out->data);
   p2.q_stride = q_out->stride[0];
-  if (launch_qproj(tw2, tl, p2, static_cast<int>(N / 128), st) != cudaSuccess) return MFA_ERR_CUDA;
+  e = launch_qproj(tw2, tl, p2, static_cast<int>(N / 128), st);
+  if (e != cudaSuccess) return cuda_fail(e);
   return MFA_OK;
 }
 
@@ -487,12 +525,15 @@ int mfa_query_proj(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor
 int mfa_read_status(mfa_stream_t stream, int reset, int* status_out) {
   if (!status_out) return MFA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MFA_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_mfa_status, sizeof v) != cudaSuccess) return MFA_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&v, g_mfa_status, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e);
   if (reset) {
     const int zero = 0;
-    if (cudaMemcpyToSymbol(g_mfa_status, &zero, sizeof zero) != cudaSuccess) return MFA_ERR_CUDA;
+    e = cudaMemcpyToSymbol(g_mfa_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   *status_out = v;
   return MFA_OK;

@@ -18,10 +18,10 @@ constexpr int kSlots = 5;                  // TMA ring slots
 constexpr int kSlotBytes = 128 * 128 * 2;  // one tensor, 128 tokens x 128 dims, bf16
 constexpr int kQBytes = kHeads * kDim * 2;
 constexpr int kPBytes = kTile * kHeads * 2;
-constexpr int kDecodeThreads = 256;        // 8 warps
+constexpr int kDecodeThreads = 384;        // 12 warps: 4 service warps + 2 softmax warpgroups
 constexpr int kTmemCols = 256;             // S0 | S1 | O_lo | O_hi, 64 columns each
 
-// One partial (split) result: O [64][256] f32 normalised over its range.
+// One partial (split) result: O [64 heads][256 d] f32, normalised over its range.
 constexpr size_t kPartialFloats = static_cast<size_t>(kHeads) * kDim;
 
 struct DecodeParams {
@@ -43,9 +43,9 @@ struct DecodeParams {
   int64_t out_sb, out_sh;  // out strides (elements) of batch and head; d stride 1
   float* lse_out;          // nullable [B][64]
   int64_t lse_sb;
-  float* ws_o;             // [slots][64][256]
-  float* ws_lse;           // [slots][64]
-  int* ws_prefix;          // [B + 1] tile prefix (balanced plan only)
+  float* ws_o;             // [slots][64 heads][256 d] normalised partial outputs
+  float* ws_lse;           // [slots][64] their log-sum-exp (natural log)
+  int* ws_prefix;          // [B + 1] first global tile of each sequence (balanced plan)
 };
 
 struct QprojParams {

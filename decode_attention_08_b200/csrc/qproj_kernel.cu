@@ -87,7 +87,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
   volatile int* abort_flag = &c.abort_flag;
-  bool acc_ok = true;
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer ----------------
@@ -110,10 +109,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t idesc = idesc_f16(128, n_cols, 1, 1, 0);
     for (int i = 0; i < nkb; ++i) {
       const int s = i % stages;
-      if (!mbar_wait(&c.full[s], (i / stages) & 1, abort_flag)) {
-        acc_ok = false;
-        break;
-      }
+      if (!mbar_wait(&c.full[s], (i / stages) & 1, abort_flag)) break;
       tc_fence_after();
       const uint32_t a = smem_u32(smem + s * stage_bytes);
       const uint32_t b = a + kABytes;
@@ -165,7 +161,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, tcols);
-  (void)acc_ok;
 
   if (p.mode == 0 && ready) {
     // deterministic split-K merge by the last CTA to finish this output tile

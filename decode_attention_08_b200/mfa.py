@@ -42,7 +42,7 @@ _lock = threading.Lock()
 
 EXPORTS = ("mfa_decode_attention", "mfa_decode_attention_ex", "mfa_decode_workspace_size",
            "mfa_query_proj", "mfa_query_proj_ex", "mfa_query_proj_workspace_size",
-           "mfa_read_status", "mfa_error_string", "mfa_version")
+           "mfa_read_status", "mfa_error_string", "mfa_version", "mfa_last_cuda_error_string")
 
 
 def lib() -> ctypes.CDLL:
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.mfa_read_status.restype = ctypes.c_int
             L.mfa_error_string.argtypes = [ctypes.c_int]
             L.mfa_error_string.restype = ctypes.c_char_p
+            L.mfa_last_cuda_error_string.argtypes = []
+            L.mfa_last_cuda_error_string.restype = ctypes.c_char_p
             L.mfa_version.argtypes = []
             L.mfa_version.restype = ctypes.c_int
             _lib = L
@@ -109,6 +111,8 @@ def _stream(stream) -> int:
 
 
 def _check(rc: int, what: str):
+    if rc == 3:
+        raise MfaError(rc, f"{what} ({lib().mfa_last_cuda_error_string().decode()})")
     if rc != 0:
         raise MfaError(rc, what)
 
@@ -141,7 +145,7 @@ def decode_attention_ex(q, k_cache, v_cache, page_table, seq_lens, out, softmax_
     """``mfa_decode_attention_ex`` (scales, split control, lse, caller workspace)."""
     need = decode_workspace_size(q.shape[0], num_splits)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     rc = lib().mfa_decode_attention_ex(
         describe(q), describe(k_cache), describe(v_cache), describe(page_table),
         describe(seq_lens), describe(out), float(softmax_scale), _kv_code(kv_dtype),

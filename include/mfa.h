@@ -110,7 +110,8 @@ int mfa_decode_attention(const mfa_tensor* q, const mfa_tensor* k_cache,
  *                    scores (-inf for empty sequences).
  *  workspace         device memory of at least
  *                    mfa_decode_workspace_size(B, num_splits) bytes, 256-byte
- *                    aligned. Contents need no initialisation.
+ *                    aligned. Contents need no initialisation. Calls that
+ *                    overlap on the GPU must not share a workspace.
  * Splitting never changes which cached rows contribute; the split plan depends
  * only on seq_lens, num_splits and the SM count, never on the cache layout, so a
  * paged and a contiguous cache holding the same rows give bit-identical results.
@@ -134,7 +135,7 @@ size_t mfa_decode_workspace_size(int batch, int num_splits);
  *  w_qa   [Dm, R] bf16 row-major (R = 2048).
  *  w_qb   [R, N] bf16 row-major (N = 64 * 256 = 16384).
  *  q_out  [B, N] bf16 (viewable as [B, 64, 256] when N = 16384).
- * 1 <= B <= 128; Dm, R multiples of 64; N a multiple of 128.
+ * 1 <= B <= 128; Dm a multiple of 64, R and N multiples of 128, R <= 131072.
  * The latent x * W_qa is accumulated in fp32 and carried into the second product
  * at about 16 significant bits (a bf16 high part plus a bf16 residual); q_out is
  * rounded once, to bf16.
@@ -159,6 +160,10 @@ int mfa_read_status(mfa_stream_t stream, int reset, int* status_out);
 
 /* Static, human-readable name of a status code. */
 const char* mfa_error_string(int code);
+
+/* Text of the CUDA error behind the most recent MFA_ERR_CUDA returned to this
+ * host thread (a static string; "no CUDA error recorded" if there was none). */
+const char* mfa_last_cuda_error_string(void);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int mfa_version(void);
