@@ -905,8 +905,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 //   out = sum_s w_s O_s / sum_s w_s,   lse = lse* + log(sum_s w_s)
 // over the sequence's partials in plan order.
 // ===========================================================================
-constexpr int kCombineHeads = 32;  // heads per CTA
-constexpr int kCombineChunk = 64;  // partial slots staged in shared memory at a time
+constexpr int kCombineHeads = 16;  // heads per CTA
 
 __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams p) {
 #ifdef MFA_TRACE
@@ -933,100 +932,74 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
     }
   } gt_end{gt_call, cta_lin};
 #endif
-  __shared__ int s_slot[kCombineChunk];
-  __shared__ float s_w[kCombineChunk][kCombineHeads];  // lse, then weights
-  __shared__ float s_m[kCombineHeads], s_l[kCombineHeads], s_scale[kCombineHeads];
   const int b = blockIdx.x;
   const int h0 = blockIdx.y * kCombineHeads;
   const int d = threadIdx.x;
 
-  const int L = valid_len(p, b);
-  const int nt = tiles_of(L);
-  if (nt == 0) {
+  SplitList sl;
+  int nt;
+  if (p.num_splits == 0) {
+    const long long S = __ldcg(p.ws_prefix + b);
+    nt = static_cast<int>(__ldcg(p.ws_prefix + b + 1) - S);
+    const long long N = __ldcg(p.ws_prefix + p.batch);
+    if (nt > 0) sl.init_balanced(S, nt, N, p.grid);
+  } else {
+    nt = tiles_of(valid_len(p, b));
+    if (nt > 0) sl.init_fixed(b, nt, p.num_splits);
+  }
+  if (nt == 0) {  // empty sequence: zeros, lse = -inf
 #pragma unroll
     for (int j = 0; j < kCombineHeads; ++j) store_out(p, b, h0 + j, d, 0.f);
     if (p.lse_out && d < kCombineHeads) p.lse_out[b * p.lse_sb + h0 + d] = -INFINITY;
     return;
   }
-  SplitList sl;
-  if (p.num_splits == 0)
-    sl.init_balanced(__ldg(p.ws_prefix + b), nt, __ldg(p.ws_prefix + p.batch), p.grid);
-  else
-    sl.init_fixed(b, nt, p.num_splits);
   if (sl.nonempty() <= 1) return;  // written directly by the attention kernel
 
-  if (d < kCombineHeads) {
-    s_m[d] = -INFINITY;
-    s_l[d] = 0.f;
+  // online merge over the partials in plan order, two slots per step:
+  // running max m, running weight sum l and running weighted sum acc per head
+  float m[kCombineHeads], l[kCombineHeads], acc[kCombineHeads];
+#pragma unroll
+  for (int j = 0; j < kCombineHeads; ++j) {
+    m[j] = -INFINITY;
+    l[j] = 0.f;
+    acc[j] = 0.f;
   }
-  float acc[kCombineHeads];
+  for (int i = 0; i < sl.count; i += 2) {
+    const int sa = sl.slot(i);
+    const int sb = i + 1 < sl.count ? sl.slot(i + 1) : -1;
+    if (sa < 0 && sb < 0) continue;
+    float la[kCombineHeads], lb[kCombineHeads], va[kCombineHeads], vb[kCombineHeads];
+    const float* oa = p.ws_o + static_cast<int64_t>(sa < 0 ? 0 : sa) * kPartialFloats +
+                      static_cast<int64_t>(h0) * kDim + d;
+    const float* ob = p.ws_o + static_cast<int64_t>(sb < 0 ? 0 : sb) * kPartialFloats +
+                      static_cast<int64_t>(h0) * kDim + d;
+    const float* ea = p.ws_lse + static_cast<int64_t>(sa < 0 ? 0 : sa) * kHeads + h0;
+    const float* eb = p.ws_lse + static_cast<int64_t>(sb < 0 ? 0 : sb) * kHeads + h0;
 #pragma unroll
-  for (int j = 0; j < kCombineHeads; ++j) acc[j] = 0.f;
-  for (int base = 0; base < sl.count; base += kCombineChunk) {
-    const int cnt = min(kCombineChunk, sl.count - base);
-    __syncthreads();
-    if (d < cnt) s_slot[d] = sl.slot(base + d);
-    __syncthreads();
-    for (int e = d; e < cnt * kCombineHeads; e += kDim) {
-      const int i = e / kCombineHeads, h = e % kCombineHeads;
-      const int sidx = s_slot[i];
-      s_w[i][h] = sidx >= 0 ? __ldcg(p.ws_lse + static_cast<int64_t>(sidx) * kHeads + h0 + h) : -INFINITY;
+    for (int j = 0; j < kCombineHeads; ++j) {
+      la[j] = sa >= 0 ? __ldcg(ea + j) : -INFINITY;
+      lb[j] = sb >= 0 ? __ldcg(eb + j) : -INFINITY;
+      va[j] = sa >= 0 ? __ldcg(oa + j * kDim) : 0.f;
+      vb[j] = sb >= 0 ? __ldcg(ob + j * kDim) : 0.f;
     }
-    __syncthreads();
-    // running max / sum per head over the chunk (online across chunks); rescale acc
-    float scale_old = 1.f;
-    if (d < kCombineHeads) {
-      const float m_old = s_m[d];
-      float m = m_old;
-      for (int i = 0; i < cnt; ++i) m = fmaxf(m, s_w[i][d]);
-      float l = s_l[d] * ex2_approx((m_old - m) * kLog2e);
-      for (int i = 0; i < cnt; ++i) {
-        const float w = ex2_approx((s_w[i][d] - m) * kLog2e);
-        s_w[i][d] = w;
-        l += w;
-      }
-      s_m[d] = m;
-      s_l[d] = l;
-      scale_old = ex2_approx((m_old - m) * kLog2e);
-    }
-    if (d < kCombineHeads) s_scale[d] = scale_old;
-    __syncthreads();
-    if (base > 0) {
 #pragma unroll
-      for (int j = 0; j < kCombineHeads; ++j) acc[j] *= s_scale[j];
-    }
-    int i = 0;
-    for (; i + 1 < cnt; i += 2) {  // two slots' loads in flight together
-      const int sa = s_slot[i], sb = s_slot[i + 1];
-      // partial layout [slot][head][d]: thread d, consecutive threads read consecutive d
-      const float* pa = p.ws_o + static_cast<int64_t>(sa < 0 ? 0 : sa) * kPartialFloats +
-                        static_cast<int64_t>(h0) * kDim + d;
-      const float* pb = p.ws_o + static_cast<int64_t>(sb < 0 ? 0 : sb) * kPartialFloats +
-                        static_cast<int64_t>(h0) * kDim + d;
-      float va[kCombineHeads], vb[kCombineHeads];
-#pragma unroll
-      for (int j = 0; j < kCombineHeads; ++j) {
-        va[j] = sa >= 0 ? __ldcg(pa + j * kDim) : 0.f;
-        vb[j] = sb >= 0 ? __ldcg(pb + j * kDim) : 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < kCombineHeads; ++j) acc[j] += s_w[i][j] * va[j] + s_w[i + 1][j] * vb[j];
-    }
-    if (i < cnt) {
-      const int sa = s_slot[i];
-      if (sa >= 0) {
-        const float* pa = p.ws_o + static_cast<int64_t>(sa) * kPartialFloats +
-                          static_cast<int64_t>(h0) * kDim + d;
-#pragma unroll
-        for (int j = 0; j < kCombineHeads; ++j) acc[j] += s_w[i][j] * __ldcg(pa + j * kDim);
-      }
+    for (int j = 0; j < kCombineHeads; ++j) {
+      const float mn = fmaxf(m[j], fmaxf(la[j], lb[j]));  // finite: one slot is valid
+      const float c = ex2_approx((m[j] - mn) * kLog2e);
+      const float wa = ex2_approx((la[j] - mn) * kLog2e);
+      const float wb = ex2_approx((lb[j] - mn) * kLog2e);
+      l[j] = l[j] * c + wa + wb;
+      acc[j] = acc[j] * c + wa * va[j] + wb * vb[j];
+      m[j] = mn;
     }
   }
-  __syncthreads();
 #pragma unroll
-  for (int j = 0; j < kCombineHeads; ++j) store_out(p, b, h0 + j, d, acc[j] / s_l[j]);
-  if (p.lse_out && d < kCombineHeads)
-    p.lse_out[b * p.lse_sb + h0 + d] = s_m[d] + lg2_approx(s_l[d]) * kLn2;
+  for (int j = 0; j < kCombineHeads; ++j) store_out(p, b, h0 + j, d, acc[j] / l[j]);
+  if (p.lse_out && d == 0) {
+#pragma unroll
+    for (int j = 0; j < kCombineHeads; ++j)
+      p.lse_out[b * p.lse_sb + h0 + j] = m[j] + lg2_approx(l[j]) * kLn2;
+  }
 }
 
 // ===========================================================================
