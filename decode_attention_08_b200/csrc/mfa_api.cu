@@ -540,3 +540,51 @@ int mfa_read_status(mfa_stream_t stream, int reset, int* status_out) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free decode attention: the split workspace lives in a fixed
+// device array owned by the library instead of memory the caller or the
+// library allocates per call.
+// ===========================================================================
+static constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(24) << 20;  // 24 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+// Device address of g_noalloc_scratch on each device, looked up on the first
+// call made with that device current (the host-side symbol is only a handle).
+void* g_noalloc_addr[kMaxDevices] = {};
+}  // namespace
+
+extern "C" int mfa_decode_attention_noalloc(const mfa_tensor* q, const mfa_tensor* k_cache,
+                                            const mfa_tensor* v_cache, const mfa_tensor* page_table,
+                                            const mfa_tensor* seq_lens, mfa_tensor* out,
+                                            float softmax_scale, int kv_dtype, float k_scale,
+                                            float v_scale, int num_splits, mfa_tensor* lse_out,
+                                            mfa_stream_t stream) {
+  const int vrc = decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale,
+                              kv_dtype, k_scale, v_scale, num_splits, lse_out, nullptr, 0, stream,
+                              true);
+  if (vrc != MFA_OK) return vrc;
+  const size_t need = mfa_decode_workspace_size(static_cast<int>(q->shape[0]), num_splits);
+  if (need == 0) return MFA_ERR_CUDA;
+  if (need > kNoAllocScratchBytes) return MFA_ERR_WORKSPACE;  // batch x splits too large
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return MFA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_noalloc_addr[dev]) {
+      e = cudaGetSymbolAddress(&g_noalloc_addr[dev], g_noalloc_scratch);
+      if (e != cudaSuccess) {
+        g_noalloc_addr[dev] = nullptr;
+        return cuda_fail(e);
+      }
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  return decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, kv_dtype,
+                     k_scale, v_scale, num_splits, lse_out, scratch, kNoAllocScratchBytes, stream,
+                     false);
+}

@@ -42,7 +42,8 @@ _lock = threading.Lock()
 
 EXPORTS = ("mfa_decode_attention", "mfa_decode_attention_ex", "mfa_decode_workspace_size",
            "mfa_query_proj", "mfa_query_proj_ex", "mfa_query_proj_workspace_size",
-           "mfa_read_status", "mfa_error_string", "mfa_version", "mfa_last_cuda_error_string")
+           "mfa_read_status", "mfa_error_string", "mfa_version", "mfa_last_cuda_error_string",
+           "mfa_decode_attention_noalloc")
 
 
 def lib() -> ctypes.CDLL:
@@ -62,6 +63,10 @@ def lib() -> ctypes.CDLL:
                                                   ctypes.c_float, ctypes.c_float, ctypes.c_int, T,
                                                   P, ctypes.c_size_t, P]
             L.mfa_decode_attention_ex.restype = ctypes.c_int
+            L.mfa_decode_attention_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_float,
+                                                       ctypes.c_int, ctypes.c_float,
+                                                       ctypes.c_float, ctypes.c_int, T, P]
+            L.mfa_decode_attention_noalloc.restype = ctypes.c_int
             L.mfa_decode_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int]
             L.mfa_decode_workspace_size.restype = ctypes.c_size_t
             L.mfa_query_proj.argtypes = [T, T, T, T, P]
@@ -152,6 +157,21 @@ def decode_attention_ex(q, k_cache, v_cache, page_table, seq_lens, out, softmax_
         float(k_scale), float(v_scale), int(num_splits), describe(lse_out),
         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "mfa_decode_attention_ex")
+    return out
+
+
+def decode_attention_noalloc(q, k_cache, v_cache, page_table, seq_lens, out,
+                             softmax_scale=1.0 / 16, kv_dtype="bf16", k_scale=1.0, v_scale=1.0,
+                             num_splits=0, lse_out=None, stream=None):
+    """``mfa_decode_attention_noalloc``: as ``decode_attention_ex`` but the split
+    workspace is the library's fixed device array, so no device memory is
+    allocated for the call (for callers that cannot allocate). Calls that
+    overlap on the GPU share that array and must be serialised."""
+    rc = lib().mfa_decode_attention_noalloc(
+        describe(q), describe(k_cache), describe(v_cache), describe(page_table),
+        describe(seq_lens), describe(out), float(softmax_scale), _kv_code(kv_dtype),
+        float(k_scale), float(v_scale), int(num_splits), describe(lse_out), _stream(stream))
+    _check(rc, "mfa_decode_attention_noalloc")
     return out
 
 

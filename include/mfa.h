@@ -128,6 +128,33 @@ int mfa_decode_attention_ex(const mfa_tensor* q, const mfa_tensor* k_cache,
 size_t mfa_decode_workspace_size(int batch, int num_splits);
 
 /*
+ * mfa_decode_attention_ex without a workspace argument and without any device
+ * allocation. The pages have no counterpart to this entry point: it is for
+ * callers that cannot allocate device memory when they call in -- for example
+ * a host framework that owns every device allocation through its own pool, or
+ * a latency-critical loop that must not pay cudaMalloc's cost and implicit
+ * device synchronisation -- and that cannot hand over a workspace either.
+ *
+ * The split workspace is a fixed 24 MiB device array inside libmfa.so, held
+ * on every device that loads the library until the process exits. Requests
+ * whose mfa_decode_workspace_size(B, num_splits) exceeds 24 MiB are rejected
+ * with MFA_ERR_WORKSPACE (on a 148-SM B200 the default balanced plan needs
+ * about 19.5 MiB plus 4 bytes per sequence; with num_splits = s the need is
+ * about 64.3 KiB per sequence and split).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. Every call on a device uses the same array and nothing
+ * in it needs to start at zero, but calls that overlap on the GPU (different
+ * streams, or different host threads) race on it: serialise them.
+ * Arguments, results and errors are otherwise those of mfa_decode_attention_ex.
+ */
+int mfa_decode_attention_noalloc(const mfa_tensor* q, const mfa_tensor* k_cache,
+                                 const mfa_tensor* v_cache, const mfa_tensor* page_table,
+                                 const mfa_tensor* seq_lens, mfa_tensor* out, float softmax_scale,
+                                 int kv_dtype, float k_scale, float v_scale, int num_splits,
+                                 mfa_tensor* lse_out, mfa_stream_t stream);
+
+/*
  * MFA low-rank query projection (Step-3 page, "Queries pass through a 2048-dim
  * low-rank bottleneck"): q_out = (x * W_qa) * W_qb, no bias, norm or activation.
  *
