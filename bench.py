@@ -367,7 +367,7 @@ def cpu_baseline(dec: gen.DecodeInputs, seconds: float):
 def other_workloads(hbm_peak: float):
     """Kernel-level numbers of the other workloads (one call per replay)."""
     res = {}
-    for idx in (1, 3, 5):
+    for idx in (1, 3, 4, 5):
         dec, proj = gen.make_workload(idx)
         big = decode_alg_bytes(dec) > L2_BYTES
         copies = 2 if big else 1

@@ -84,6 +84,7 @@ struct __align__(16) DecodeCtrl {
   uint64_t slot_full[kSlots], slot_empty[kSlots];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, o_full;
+  uint64_t conv_full[kSlots], q_conv;  // FP8 cache: ring slot / q expanded to f16
   uint64_t red_full[kWG][2], l_full[kWG];
   uint64_t drain;
   long long t0;    // first global tile of this CTA (balanced plan)
@@ -428,12 +429,79 @@ __device__ __forceinline__ uint32_t v_item(uint32_t j, bool cta_last) {
   return cta_last ? 4u * j + 2u : 4u * j + 4u;
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// two E4M3 codes (low byte = first element) -> f16x2, exact
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t out;
+  const uint16_t in = static_cast<uint16_t>(two_codes);
+  asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(out)
+      : "h"(in));
+  return out;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// FP8 cache: expand one ring slot in place. TMA wrote an E4M3 half-tile of 128
+// token rows x 128 head dims (128-byte rows, 128-byte swizzle) into the slot's
+// first 16 KB; it becomes the f16 half-tile the MMA reads: two 16 KB regions
+// (dims 0-63, 64-127) of 128-byte swizzled rows. Each lane owns whole rows: it
+// reads its row completely before writing, and region 0's row r sits exactly on
+// input row r, so no row is overwritten before it has been read.
+__device__ __forceinline__ void expand_fp8_halftile(uint32_t base, int lane) {
+#pragma unroll 1
+  for (int row = lane; row < kTile; row += 32) {
+    const uint32_t in = base + row * 128;
+    const int sw = row & 7;
+    uint4 v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) v[c] = ld_shared_v4(in + ((c ^ sw) << 4));
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {  // input chunk c = dims 16c..16c+15
+      const uint32_t dst = base + (c >> 2) * (kSlotBytes / 2) + row * 128;
+      const int c2 = (c & 3) * 2;
+      st_shared_v4(dst + ((c2 ^ sw) << 4), e4m3x2_to_f16x2(v[c].x),
+                   e4m3x2_to_f16x2(v[c].x >> 16), e4m3x2_to_f16x2(v[c].y),
+                   e4m3x2_to_f16x2(v[c].y >> 16));
+      st_shared_v4(dst + (((c2 + 1) ^ sw) << 4), e4m3x2_to_f16x2(v[c].z),
+                   e4m3x2_to_f16x2(v[c].z >> 16), e4m3x2_to_f16x2(v[c].w),
+                   e4m3x2_to_f16x2(v[c].w >> 16));
+    }
+  }
+}
+
+// FP8 cache: q (bf16, 32 KB) to f16 in place, for f16 x f16 MMAs.
+__device__ __forceinline__ void q_to_f16(uint32_t base, int lane) {
+#pragma unroll 4
+  for (int i = lane; i < kQBytes / 16; i += 32) {
+    uint4 v = ld_shared_v4(base + i * 16);
+    st_shared_v4(base + i * 16, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                 bf16x2_to_f16x2(v.w));
+  }
+}
+
 }  // namespace
 
 // ===========================================================================
 // the attention kernel
 // ===========================================================================
-template <bool kPaged>
+template <bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     mfa_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -475,6 +543,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     mbar_init(&c.p_full, 4 * kWG);
     mbar_init(&c.o_full, 1);
+    for (int i = 0; i < kSlots; ++i) mbar_init(&c.conv_full[i], 1);
+    mbar_init(&c.q_conv, 1);
     mbar_init(&c.drain, 1);
     c.abort_flag = 0;
     c.b_start = 0;
@@ -537,18 +607,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           if (half == 0) MFA_TR(kind, ntr[kind]);
           uint8_t* dst = sRing + slot * kSlotBytes;
           const int t0 = t.tile * kTile;
+          // bf16: two boxes of 64 dims x 128 rows; FP8: one box of 128 dims x 128
+          // rows into the slot's first half (expanded to f16 by the converter)
+          constexpr int kBoxes = kFp8 ? 1 : 2;
+          constexpr int kBoxDims = kFp8 ? 128 : 64;
           if (!kPaged) {
-            mbar_arrive_expect_tx(&c.slot_full[slot], kSlotBytes);
-            for (int r = 0; r < 2; ++r)
+            mbar_arrive_expect_tx(&c.slot_full[slot], kFp8 ? kSlotBytes / 2 : kSlotBytes);
+            for (int r = 0; r < kBoxes; ++r)
               tma_load_3d(dst + r * (kSlotBytes / 2), map, &c.slot_full[slot],
-                          (2 * half + r) * 64, t0, t.b, policy);
+                          (kBoxes * half + r) * kBoxDims, t0, t.b, policy);
           } else {
             const int ps = p.page_size;
             const int rows = ps < kTile ? ps : kTile;
             const int nsub = kTile / rows;
             uint32_t bytes = 0;
             for (int j = 0; j < nsub; ++j)
-              if (t0 + j * rows < t.L) bytes += rows * 128 * 2;
+              if (t0 + j * rows < t.L) bytes += rows * 128 * kBoxes;
             mbar_arrive_expect_tx(&c.slot_full[slot], bytes);
             for (int j = 0; j < nsub; ++j) {
               const int tok = t0 + j * rows;
@@ -558,9 +632,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                 record_error(5 /* MFA_ERR_BAD_INDEX */);
                 phys = 0;
               }
-              for (int r = 0; r < 2; ++r)
+              for (int r = 0; r < kBoxes; ++r)
                 tma_load_3d(dst + r * (kSlotBytes / 2) + j * rows * 128, map, &c.slot_full[slot],
-                            (2 * half + r) * 64, tok % ps, phys, policy);
+                            (kBoxes * half + r) * kBoxDims, tok % ps, phys, policy);
             }
           }
         }
@@ -585,8 +659,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =====================================
-    constexpr uint32_t idesc_qk = idesc_f16(128, 64, 1, 0, 0);
-    constexpr uint32_t idesc_pv = idesc_f16(128, 64, 1, 1, 1);
+    // operands: bf16 for a bf16 cache; f16 (exact expansion of E4M3, q and P in
+    // f16) for an FP8 cache
+    constexpr int kAB = kFp8 ? 0 : 1;
+    constexpr uint32_t idesc_qk = idesc_f16(128, 64, kAB, 0, 0);
+    constexpr uint32_t idesc_pv = idesc_f16(128, 64, kAB, 1, 1);
+    uint64_t* operand_ready = kFp8 ? c.conv_full : c.slot_full;
     const uint32_t q_base = smem_u32(sQ);
     const uint32_t ring_base = smem_u32(sRing);
     const uint32_t p_base = smem_u32(sP);
@@ -598,8 +676,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     auto issue_pv = [&](const TileInfo& t, uint32_t j) -> bool {
       if (!warp_wait(&c.p_full, par(j), abort_flag)) return false;
       const uint32_t lo = item++, hi = item++;
-      if (!warp_wait(&c.slot_full[lo % kSlots], par(lo / kSlots), abort_flag)) return false;
-      if (!warp_wait(&c.slot_full[hi % kSlots], par(hi / kSlots), abort_flag)) return false;
+      if (!warp_wait(&operand_ready[lo % kSlots], par(lo / kSlots), abort_flag)) return false;
+      if (!warp_wait(&operand_ready[hi % kSlots], par(hi / kSlots), abort_flag)) return false;
       tc_fence_after();
       if (lane == 0) {
         MFA_TR(3, j);
@@ -628,14 +706,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     uint32_t g = 0;
     while (ok && qs.next(cur)) {
       if (cur.seg_first) {
-        ok = warp_wait(&c.q_full, par(nq), abort_flag);
+        ok = warp_wait(kFp8 ? &c.q_conv : &c.q_full, par(nq), abort_flag);
         ++nq;
         if (!ok) break;
       }
       if (g >= 2 && !(ok = warp_wait(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag))) break;
       const uint32_t lo = item++, hi = item++;
-      if (!(ok = warp_wait(&c.slot_full[lo % kSlots], par(lo / kSlots), abort_flag))) break;
-      if (!(ok = warp_wait(&c.slot_full[hi % kSlots], par(hi / kSlots), abort_flag))) break;
+      if (!(ok = warp_wait(&operand_ready[lo % kSlots], par(lo / kSlots), abort_flag))) break;
+      if (!(ok = warp_wait(&operand_ready[hi % kSlots], par(hi / kSlots), abort_flag))) break;
       tc_fence_after();
       if (lane == 0) {
         MFA_TR(2, g);
@@ -692,6 +770,41 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         for (int r = 0; r < 4; ++r) tma_prefetch_3d(&tm_q, r * 64, 0, ta.b);
       __syncwarp();
       ++k;
+    }
+  } else if (warp == 3) {
+    // ======================= FP8 converter ==================================
+    // Follows the MMA's consumption order: q at each segment start, then K of
+    // tile g and V of tile g-1, each half-tile expanded in place to f16.
+    if (kFp8) {
+      TileStream cs;
+      cs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+      uint32_t item = 0, nq = 0, g = 0;
+      auto convert_item = [&]() -> bool {
+        const uint32_t slot = item % kSlots;
+        if (!warp_wait(&c.slot_full[slot], par(item / kSlots), abort_flag)) return false;
+        expand_fp8_halftile(smem_u32(sRing + slot * kSlotBytes), lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.conv_full[slot]);
+        ++item;
+        return true;
+      };
+      TileInfo t;
+      bool ok = true;
+      while (ok && cs.next(t)) {
+        if (t.seg_first) {
+          if (!(ok = warp_wait(&c.q_full, par(nq), abort_flag))) break;
+          q_to_f16(smem_u32(sQ), lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.q_conv);
+          ++nq;
+        }
+        ok = convert_item() && convert_item();             // K of tile g
+        if (ok && g >= 1) ok = convert_item() && convert_item();  // V of tile g-1
+        ++g;
+      }
+      if (ok && g >= 1) ok = convert_item() && convert_item();    // V of the last tile
     }
   } else if (warp >= 4) {
     // ======================= softmax + epilogue =============================
@@ -781,8 +894,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           l_part[h + 2] += p2;
           l_part[h + 3] += p3;
         }
-        pk[h / 2] = pack_bf16x2(p0, p1);
-        pk[h / 2 + 1] = pack_bf16x2(p2, p3);
+        pk[h / 2] = kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+        pk[h / 2 + 1] = kFp8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
       }
 
       // ---- P buffer and O are free once the previous tile's PV completed --
@@ -814,7 +927,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // reaches the accumulator (warpgroup 0: head dims 0-127, 1: 128-255)
       if (valid < kTile) {
         const uint32_t it = v_item(g, t.cta_last) + wg;
-        if (!warp_wait(&c.slot_full[it % kSlots], par(it / kSlots), abort_flag)) break;
+        uint64_t* ready = kFp8 ? c.conv_full : c.slot_full;  // zero after the FP8 expansion
+        if (!warp_wait(&ready[it % kSlots], par(it / kSlots), abort_flag)) break;
         if (!row_ok) {
           const uint32_t base = smem_u32(sRing) + (it % kSlots) * kSlotBytes + row * 128;
 #pragma unroll
@@ -1023,24 +1137,32 @@ static cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-cudaError_t launch_decode(bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
-                          const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
-  static thread_local int configured_dev[2] = {-1, -1};
+template <bool kPaged, bool kFp8>
+static cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk,
+                                    const CUtensorMap& tv, const DecodeParams& p,
+                                    cudaStream_t stream) {
+  static thread_local int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
-  cudaError_t err;
-  if (configured_dev[paged ? 1 : 0] != dev) {
-    err = paged ? cudaFuncSetAttribute(mfa_decode_kernel<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)
-                : cudaFuncSetAttribute(mfa_decode_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (configured_dev != dev) {
+    const cudaError_t err = cudaFuncSetAttribute(
+        mfa_decode_kernel<kPaged, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
-    configured_dev[paged ? 1 : 0] = dev;
+    configured_dev = dev;
   }
-  err = paged ? launch_pdl(mfa_decode_kernel<true>, dim3(p.grid), dim3(kDecodeThreads),
-                           kSmemBytes, stream, tq, tk, tv, p)
-              : launch_pdl(mfa_decode_kernel<false>, dim3(p.grid), dim3(kDecodeThreads),
-                           kSmemBytes, stream, tq, tk, tv, p);
+  return launch_pdl(mfa_decode_kernel<kPaged, kFp8>, dim3(p.grid), dim3(kDecodeThreads),
+                    kSmemBytes, stream, tq, tk, tv, p);
+}
+
+cudaError_t launch_decode(bool paged, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
+                          const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
+  cudaError_t err;
+  if (fp8)
+    err = paged ? launch_attention<true, true>(tq, tk, tv, p, stream)
+                : launch_attention<false, true>(tq, tk, tv, p, stream);
+  else
+    err = paged ? launch_attention<true, false>(tq, tk, tv, p, stream)
+                : launch_attention<false, false>(tq, tk, tv, p, stream);
   if (err != cudaSuccess) return err;
   return launch_pdl(mfa_combine_kernel, dim3(p.batch, kHeads / kCombineHeads), dim3(kDim), 0,
                     stream, p);

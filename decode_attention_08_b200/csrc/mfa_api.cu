@@ -12,7 +12,7 @@
 
 namespace mfa {
 int decode_smem_bytes();
-cudaError_t launch_decode(bool paged, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_decode(bool paged, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                           const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);
 int qproj_smem_bytes(int n_cols);
 cudaError_t launch_qproj(const CUtensorMap& tw, const CUtensorMap& ta, const QprojParams& p,
@@ -288,8 +288,9 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
   if (q->stride[2] != 1 || q->stride[1] % 8 || q->stride[0] % 8) return MFA_ERR_INVALID_ARG;
   if (kv_dtype != MFA_BF16 && kv_dtype != MFA_FP8_E4M3) return MFA_ERR_INVALID_ARG;
   if (k_cache->dtype != kv_dtype || v_cache->dtype != kv_dtype) return MFA_ERR_INVALID_ARG;
-  if (kv_dtype == MFA_FP8_E4M3) return MFA_ERR_UNSUPPORTED;  // FP8 path: see decode_fp8
   if (kv_dtype == MFA_BF16 && (k_scale != 1.f || v_scale != 1.f)) return MFA_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || k_scale > 1e30f || v_scale > 1e30f)
+    return MFA_ERR_INVALID_ARG;
   for (int i = 0; i < 3; ++i)
     if (k_cache->shape[i] != v_cache->shape[i]) return MFA_ERR_INVALID_ARG;
   if (k_cache->shape[2] != kDim) return MFA_ERR_UNSUPPORTED;
@@ -355,10 +356,15 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
     // a zero-length cache: nothing is ever loaded, but a map needs extent >= 1
   }
   const uint64_t d1s = d1 > 0 ? d1 : 1;
-  if (encode_3d(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_cache->data, kDim, d1s, d2,
-                k_cache->stride[1], k_cache->stride[0], 64, rows) != CUDA_SUCCESS ||
-      encode_3d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v_cache->data, kDim, d1s, d2,
-                v_cache->stride[1], v_cache->stride[0], 64, rows) != CUDA_SUCCESS)
+  // bf16: boxes of 64 dims (128 bytes); E4M3: boxes of 128 dims (128 bytes)
+  const bool fp8 = kv_dtype == MFA_FP8_E4M3;
+  const CUtensorMapDataType kv_type =
+      fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint32_t box0 = fp8 ? 128 : 64;
+  if (encode_3d(&tk, kv_type, esz, k_cache->data, kDim, d1s, d2, k_cache->stride[1],
+                k_cache->stride[0], box0, rows) != CUDA_SUCCESS ||
+      encode_3d(&tv, kv_type, esz, v_cache->data, kDim, d1s, d2, v_cache->stride[1],
+                v_cache->stride[0], box0, rows) != CUDA_SUCCESS)
     return MFA_ERR_INVALID_ARG;
 
   DecodeParams p;
@@ -387,7 +393,8 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
   p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
   p.ws_prefix = reinterpret_cast<int*>(ws + wl.prefix_off);
 
-  const cudaError_t err = launch_decode(paged, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t err =
+      launch_decode(paged, fp8, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? MFA_OK : cuda_fail(err);
 }
 
