@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle's CPU-baseline sample")
-    ap.add_argument("--profile", choices=["decode", "paged", "qproj"], default=None,
+    ap.add_argument("--profile", choices=["decode", "paged", "fp8", "qproj"], default=None,
                     help="profiling case for ncu: plain launches of one kernel family on a "
                          "reduced workload that still exceeds L2")
     return ap.parse_args()
@@ -72,12 +72,22 @@ def dist_setup(gpus: int):
     return world, rank, local
 
 
+def _dist_device() -> str:
+    return "cpu" if torch.distributed.get_backend() == "gloo" else "cuda"
+
+
 def dist_max(x: float, world: int) -> float:
+    """Max over ranks of a per-rank elapsed time (the only cross-rank reduction)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_dist_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank_step: int, steps: int, world: int, t_max: float) -> float:
+    """Whole-job throughput: units every rank processed over the slowest rank's time."""
+    return units_per_rank_step * steps * world / t_max
 
 
 def barrier(world: int):
@@ -462,7 +472,7 @@ def run_ours(args, world, rank, local):
     t_max = dist_max(secs, world)
 
     T = dec.total_tokens
-    value = T * args.steps * world / t_max
+    value = weak_scaling_value(T, args.steps, world, t_max)
     per_launch = secs / args.steps
     alg = decode_alg_bytes(dec)
     achieved = alg / per_launch / 1e9
@@ -561,6 +571,8 @@ def run_profile_case(args):
     else:
         if args.profile == "decode":
             dec = gen.make_decode_inputs(1002, 48, 4096)
+        elif args.profile == "fp8":
+            dec = gen.make_decode_inputs(1004, 96, 4096, kv_dtype="e4m3")
         else:
             lens = gen.workload_lengths(3)[:40].tolist()
             dec = gen.make_decode_inputs(1003, 40, lens, page_size=64)
