@@ -45,7 +45,7 @@ namespace mfa {
 // Optional pipeline trace (compile with -DMFA_TRACE; off in the library build):
 // clock64() stamps of pipeline events for the first 64 tiles of each CTA.
 #ifdef MFA_TRACE
-constexpr int kTraceKinds = 12, kTraceTiles = 64, kTraceCtas = 160;
+constexpr int kTraceKinds = 16, kTraceTiles = 64, kTraceCtas = 160;
 __device__ unsigned long long g_mfa_trace[kTraceCtas * kTraceKinds * kTraceTiles];
 #define MFA_TR(kind, idx)                                                                   \
   do {                                                                                      \
@@ -131,11 +131,6 @@ __device__ __forceinline__ int valid_len(const DecodeParams& p, int b) {
   return L;
 }
 
-// Sequence length: from the block's shared copy when the batch fits in it.
-__device__ __forceinline__ int seq_len(const DecodeParams& p, const int* lens, int b) {
-  return lens ? lens[b] : valid_len(p, b);
-}
-
 // All lanes wait; the outcome is made warp-uniform.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const bool ok = mbar_wait(bar, parity, abort);
@@ -160,8 +155,12 @@ struct TileInfo {
 };
 
 struct TileStream {
-  const DecodeParams* p;
+  // scalars copied out of the parameter block at init, so walking the stream
+  // never reloads them through memory (the hot loops hold memory-clobbering
+  // waits, after which a pointer read would go back out to the cache hierarchy)
+  const int* seq_lens;
   const int* lens;  // shared copy of the lengths, or nullptr
+  int cap_tokens, num_splits, grid, batch;
   int cta;
   int b, tile, L, nt, remaining, seg_lo, seg_hi, seg_ord;
   long long gtile;
@@ -169,8 +168,12 @@ struct TileStream {
 
   __device__ void init(const DecodeParams& prm, const int* lens_, int b_start, int off_start,
                        int tiles, long long t0) {
-    p = &prm;
+    seq_lens = prm.seq_lens;
     lens = lens_;
+    cap_tokens = prm.cap_tokens;
+    num_splits = prm.num_splits;
+    grid = prm.grid;
+    batch = prm.batch;
     cta = blockIdx.x;
     seg_ord = 0;
     gtile = t0;
@@ -178,7 +181,7 @@ struct TileStream {
       remaining = tiles;
       if (remaining > 0) {
         b = b_start;
-        L = seq_len(prm, lens, b);
+        L = length(b);
         nt = tiles_of(L);
         tile = off_start;
         seg_lo = tile;
@@ -192,13 +195,23 @@ struct TileStream {
   }
 
   // fixed plan: move to the next non-empty unit owned by this CTA
+  __device__ int length(int seq) const {
+    if (lens) return lens[seq];
+    int n = __ldg(seq_lens + seq);
+    if (n < 0 || n > cap_tokens) {
+      record_error(5 /* MFA_ERR_BAD_INDEX */);
+      n = 0;
+    }
+    return n;
+  }
+
   __device__ void advance_unit() {
-    const int s = p->num_splits;
-    const int nunits = p->batch * s;
-    for (unit += p->grid; unit < nunits; unit += p->grid) {
+    const int s = num_splits;
+    const int nunits = batch * s;
+    for (unit += grid; unit < nunits; unit += grid) {
       b = unit / s;
       const int j = unit % s;
-      L = seq_len(*p, lens, b);
+      L = length(b);
       nt = tiles_of(L);
       const int lo = static_cast<int>((static_cast<long long>(j) * nt) / s);
       const int hi = static_cast<int>((static_cast<long long>(j + 1) * nt) / s);
@@ -223,7 +236,7 @@ struct TileStream {
     t.seg_last = (tile == seg_hi - 1);
     t.gtile = gtile;
     const bool complete = (seg_lo == 0 && seg_hi == nt);
-    if (p->num_splits == 0) {
+    if (num_splits == 0) {
       t.slot = complete ? -1 : (2 * cta + (seg_ord == 0 ? 0 : 1));
       ++tile;
       ++gtile;
@@ -232,7 +245,7 @@ struct TileStream {
       if (remaining > 0 && tile == nt) {
         do {
           ++b;
-          L = seq_len(*p, lens, b);
+          L = length(b);
           nt = tiles_of(L);
         } while (nt == 0);
         tile = 0;
@@ -429,6 +442,26 @@ __device__ __forceinline__ uint32_t v_item(uint32_t j, bool cta_last) {
   return cta_last ? 4u * j + 2u : 4u * j + 4u;
 }
 
+// Page ids of 32 consecutive logical pages of one sequence, one per lane of the
+// producer warp, so a TMA issue never waits on a dependent page-table load:
+// a refill reads up to 32 entries in parallel (never past the sequence's last
+// page, as the interface promises) and ids are taken by warp shuffle.
+struct PageWindow {
+  int b = -1, base = 0, val = 0;
+  // id of logical page `lp` (per lane) of sequence `seq`; [lo, hi] (warp-uniform,
+  // hi - lo < 32) bounds the pages the warp asks for in this call
+  __device__ __forceinline__ int get(const int* table, int64_t stride, int seq, int lo, int hi,
+                                     int lp, int npages, int lane) {
+    if (seq != b || lo < base || hi >= base + 32) {  // warp-uniform
+      b = seq;
+      base = lo;
+      const int mine = base + lane;
+      val = mine < npages ? __ldg(table + static_cast<int64_t>(seq) * stride + mine) : 0;
+    }
+    return __shfl_sync(0xffffffffu, val, lp - base);
+  }
+};
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -593,69 +626,120 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   } else if (warp == 0) {
     // ======================= K/V producer ===================================
     const uint64_t policy = l2_policy_evict_first();
-    TileStream ks, vs;
+    TileStream ks;
     ks.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
-    vs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
     uint32_t item = 0;
+#ifdef MFA_TRACE
     int ntr[2] = {0, 0};
-    auto load = [&](const TileInfo& t, const CUtensorMap* map) -> bool {
-      const int kind = (map == &tm_k) ? 0 : 1;
-      for (int half = 0; half < 2; ++half) {
-        const uint32_t slot = item % kSlots;
-        if (!warp_wait(&c.slot_empty[slot], par(item / kSlots) ^ 1u, abort_flag)) return false;
-        if (lane == 0) {
-          if (half == 0) MFA_TR(kind, ntr[kind]);
+#endif
+    PageWindow win;
+    // paged-cache fields held in registers for the whole loop; page sizes are
+    // powers of two, so every page split is a shift or a mask
+    const int ps = kPaged ? p.page_size : kTile;
+    const int pshift = __ffs(ps) - 1;
+    const int rshift = pshift < 7 ? pshift : 7;  // log2 tokens per box (one page, or one tile)
+    const int rows = 1 << rshift;
+    const int nsub = kTile >> rshift;
+    const int num_pages = p.num_pages;
+    const int* page_table = p.page_table;
+    const int64_t pt_stride = p.pt_stride;
+    // bf16: two boxes of 64 dims x rows per half (or one 4-D box of both);
+    // FP8: one box of 128 dims into the slot's first half, expanded to f16 by
+    // the converter
+    constexpr int kBoxes = kFp8 ? 1 : 2;
+    constexpr int kBoxDims = kFp8 ? 128 : 64;
+    const bool four_d = !kFp8 && rshift == 7;  // contiguous bf16, or bf16 pages >= 128
+
+    // Sub-pages of a tile (paged caches): lane j < nbox loads sub-page j (a
+    // page, or the part of a >= 128-token page under the tile) and holds its
+    // page id. K and V share the page table, so a tile is looked up once.
+    auto lookup = [&](const TileInfo& t, int& page, int& nbox) {
+      page = 0;
+      nbox = 1;
+      if (kPaged) {
+        const int t0 = t.tile * kTile;
+        const int live = (t.L - t0 + rows - 1) >> rshift;
+        nbox = live < nsub ? live : nsub;
+        const int first = t0 >> pshift;
+        page = win.get(page_table, pt_stride, t.b, first, first + nbox - 1,
+                       first + (lane < nbox ? lane : 0), (t.L + ps - 1) >> pshift, lane);
+        if (lane < nbox && (page < 0 || page >= num_pages)) {
+          record_error(5 /* MFA_ERR_BAD_INDEX */);
+          page = 0;
+        }
+      }
+    };
+    // The producer's steady-state code is kept to one short copy (K and V go
+    // through the same issue site): it runs seldom next to the consumers' hot
+    // loops, so each instruction-cache line it touches tends to be refetched
+    // from L2, slowly while HBM is saturated.
+    TileInfo tk, tv;       // the next K tile; the tile whose V is pending
+    int pgk = 0, nbk = 1;  // lookups of tk
+    int pgv = 0, nbv = 1;  // lookups of tv
+    bool have_k = ks.next(tk), have_v = false;
+    if (have_k) lookup(tk, pgk, nbk);
+    // ring order K0 K1 V0 K2 V1 ... K(T-1) V(T-2) V(T-1): round i issues K_i
+    // (phase 0), then V_(i-1) (phase 1), then moves to the next tile
+    int phase = 0;
+    while (have_k || have_v) {
+      const bool is_k = phase == 0;
+      if (is_k ? have_k : have_v) {
+        const TileInfo t = is_k ? tk : tv;
+        const int page = is_k ? pgk : pgv;
+        const int nbox = is_k ? nbk : nbv;
+        const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+        const int kind = is_k ? 0 : 1;
+        const int t0 = t.tile * kTile;
+        const uint32_t bytes =
+            four_d ? kSlotBytes : static_cast<uint32_t>(nbox * rows * 128 * kBoxes);
+        bool ok = true;
+        for (int half = 0; half < 2 && ok; ++half) {
+          const uint32_t slot = item % kSlots;
+          ok = warp_wait(&c.slot_empty[slot], par(item / kSlots) ^ 1u, abort_flag);
+          if (!ok) break;
           uint8_t* dst = sRing + slot * kSlotBytes;
-          const int t0 = t.tile * kTile;
-          // bf16: two boxes of 64 dims x 128 rows; FP8: one box of 128 dims x 128
-          // rows into the slot's first half (expanded to f16 by the converter)
-          constexpr int kBoxes = kFp8 ? 1 : 2;
-          constexpr int kBoxDims = kFp8 ? 128 : 64;
-          if (!kPaged) {
-            mbar_arrive_expect_tx(&c.slot_full[slot], kFp8 ? kSlotBytes / 2 : kSlotBytes);
-            for (int r = 0; r < kBoxes; ++r)
-              tma_load_3d(dst + r * (kSlotBytes / 2), map, &c.slot_full[slot],
-                          (kBoxes * half + r) * kBoxDims, t0, t.b, policy);
-          } else {
-            const int ps = p.page_size;
-            const int rows = ps < kTile ? ps : kTile;
-            const int nsub = kTile / rows;
-            uint32_t bytes = 0;
-            for (int j = 0; j < nsub; ++j)
-              if (t0 + j * rows < t.L) bytes += rows * 128 * kBoxes;
+          if (lane == 0) {
+            if (half == 0) MFA_TR(kind, ntr[kind]);
             mbar_arrive_expect_tx(&c.slot_full[slot], bytes);
-            for (int j = 0; j < nsub; ++j) {
-              const int tok = t0 + j * rows;
-              if (tok >= t.L) break;
-              int phys = __ldg(p.page_table + static_cast<int64_t>(t.b) * p.pt_stride + tok / ps);
-              if (phys < 0 || phys >= p.num_pages) {
-                record_error(5 /* MFA_ERR_BAD_INDEX */);
-                phys = 0;
-              }
+          }
+          __syncwarp();
+          if (lane < nbox) {
+            const int outer = kPaged ? page : t.b;
+            if (four_d) {
+              // the map views each token row as 4 chunks of 64 dims (chunk
+              // stride 128 B) after the token dimension: the box lands as
+              // [chunk][128 tokens][128 B]
+              tma_load_4d(dst, map, &c.slot_full[slot], 0, kPaged ? (t0 & (ps - 1)) : t0,
+                          2 * half, outer, policy);
+            } else {
+              const int tok = t0 + (lane << rshift);
               for (int r = 0; r < kBoxes; ++r)
-                tma_load_3d(dst + r * (kSlotBytes / 2) + j * rows * 128, map, &c.slot_full[slot],
-                            (kBoxes * half + r) * kBoxDims, tok % ps, phys, policy);
+                tma_load_3d(dst + r * (kSlotBytes / 2) + lane * rows * 128, map,
+                            &c.slot_full[slot], (kBoxes * half + r) * kBoxDims,
+                            kPaged ? (tok & (ps - 1)) : tok, outer, policy);
             }
           }
+          __syncwarp();
+          ++item;
         }
-        __syncwarp();
-        ++item;
+        if (!ok) break;
+#ifdef MFA_TRACE
+        if (lane == 0) MFA_TR(14 + kind, ntr[kind]);  // both halves issued
+        ++ntr[kind];
+#endif
       }
-      ++ntr[kind];
-      return true;
-    };
-    TileInfo kt, vt;
-    bool more_k = ks.next(kt);
-    bool first = true, ok = true;
-    while (ok) {
-      if (more_k) ok = load(kt, &tm_k);
-      if (ok && !first) {
-        vs.next(vt);
-        ok = load(vt, &tm_v);
+      if (!is_k) {
+        // end of the round: this K tile's V is next; fetch the following K tile
+        have_v = have_k;
+        if (have_k) {
+          tv = tk;
+          pgv = pgk;
+          nbv = nbk;
+          have_k = ks.next(tk);
+          if (have_k) lookup(tk, pgk, nbk);
+        }
       }
-      if (!more_k) break;
-      first = false;
-      more_k = ks.next(kt);
+      phase ^= 1;
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =====================================
