@@ -91,6 +91,7 @@ struct __align__(16) DecodeCtrl {
   long long ntot;  // total tiles of the batch (balanced plan)
   uint32_t tmem_base;
   int abort_flag;
+  unsigned seg_arrivals;  // bf16 cache: softmax-warp arrivals at segment ends (never wraps)
   int b_start, off_start, tiles;
   int scan_warp[kDecodeThreads / 32];
   int lens[kDecodeThreads];  // validated seq_lens when batch <= kDecodeThreads
@@ -99,6 +100,7 @@ struct __align__(16) DecodeCtrl {
   alignas(16) float mv[kWG][4][kWGHeads];      // per-warp copy: running max in use
   alignas(16) float cv[kWG][4][kWGHeads];      // per-warp copy: rescale factors / out scale
   alignas(16) float lred[kWG][4][kWGHeads];    // per-warp partial row sums (epilogue)
+  alignas(16) float ev[kWG][4][kWGHeads];      // per-warp copy: output scale of a segment
 };
 static_assert(offsetof(DecodeCtrl, red) % 16 == 0 && offsetof(DecodeCtrl, mv) % 16 == 0 &&
                   offsetof(DecodeCtrl, cv) % 16 == 0 && offsetof(DecodeCtrl, lred) % 16 == 0,
@@ -115,6 +117,9 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kColS = 0;      // two 64-column score buffers
 constexpr uint32_t kColOlo = 128;  // O^T rows 0..127
 constexpr uint32_t kColOhi = 192;  // O^T rows 128..255
+constexpr uint32_t kColObuf = 256; // column offset of the odd segments' O pair
+
+__device__ __forceinline__ uint32_t o_cols(int seg) { return (seg & 1) ? kColObuf : 0u; }
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -151,6 +156,7 @@ struct TileInfo {
   bool seg_last;    // last tile of a segment
   bool cta_last;    // last tile this CTA processes
   int slot;         // partial slot of the segment, -1 when it covers the sequence
+  int seg;          // ordinal of the segment among this CTA's segments
   long long gtile;  // global tile index (balanced plan)
 };
 
@@ -163,6 +169,7 @@ struct TileStream {
   int cap_tokens, num_splits, grid, batch;
   int cta;
   int b, tile, L, nt, remaining, seg_lo, seg_hi, seg_ord;
+  int segno;  // segments completed so far
   long long gtile;
   int unit, unit_hi;
 
@@ -176,6 +183,7 @@ struct TileStream {
     batch = prm.batch;
     cta = blockIdx.x;
     seg_ord = 0;
+    segno = 0;
     gtile = t0;
     if (prm.num_splits == 0) {
       remaining = tiles;
@@ -234,6 +242,8 @@ struct TileStream {
     t.L = L;
     t.seg_first = (tile == seg_lo);
     t.seg_last = (tile == seg_hi - 1);
+    t.seg = segno;
+    if (t.seg_last) ++segno;
     t.gtile = gtile;
     const bool complete = (seg_lo == 0 && seg_hi == nt);
     if (num_splits == 0) {
@@ -314,6 +324,81 @@ struct SplitList {
   }
 };
 
+// Partial slots (segments) of the tile's sequence under the plan in use.
+__device__ __forceinline__ int segments_of(const DecodeParams& p, const TileInfo& t,
+                                           long long ntot) {
+  SplitList sl;
+  if (p.num_splits == 0) {
+    sl.init_balanced(t.gtile - t.tile, tiles_of(t.L), ntot, p.grid);
+    return sl.count;
+  }
+  sl.init_fixed(t.b, tiles_of(t.L), p.num_splits);
+  return sl.nonempty();
+}
+
+__device__ __forceinline__ void smem_add_release(unsigned* ctr, unsigned v) {
+  asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(ctr)), "r"(v)
+               : "memory");
+}
+
+__device__ __forceinline__ unsigned smem_ld_acquire(const unsigned* ctr) {
+  unsigned v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(ctr)) : "memory");
+  return v;
+}
+
+// Waits (bounded, like mbar_wait) until the shared counter reaches `target`.
+__device__ __forceinline__ bool wait_count(const unsigned* ctr, unsigned target,
+                                           volatile int* abort_flag) {
+  if (smem_ld_acquire(ctr) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (smem_ld_acquire(ctr) >= target) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        record_error(6 /* MFA_ERR_TIMEOUT */);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// the four ready words of a sequence (32 bytes, 16-byte aligned)
+__device__ __forceinline__ void st_ready4(unsigned long long* dst, unsigned long long v) {
+  asm volatile(
+      "st.volatile.global.v2.b64 [%0], {%1, %1};\n\t"
+      "st.volatile.global.v2.b64 [%0+16], {%1, %1};" ::"l"(dst),
+      "l"(v)
+      : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* src) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(src) : "memory");
+  return v;
+}
+
+// Publishes the end of a segment to the combine kernel (one thread). For a
+// split sequence the call counts as one of `arrivals` x (segments) arrivals;
+// the last one (after whose arrival every partial is in memory: each arriver
+// made its partial visible first) sets the ready words to "merge". A sequence
+// that one segment covers is marked "nothing to merge".
+__device__ __forceinline__ void publish_segment(const DecodeParams& p, const TileInfo& t,
+                                                long long ntot, unsigned arrivals) {
+  unsigned long long word = kReadyNone;
+  if (t.slot >= 0) {
+    __threadfence();  // the partial (made visible to this thread) before the arrival
+    const unsigned n = arrivals * static_cast<unsigned>(segments_of(p, t, ntot));
+    if (atomicInc(p.ws_arrive + t.b, n - 1) != n - 1) return;  // wraps to 0 on the last
+    __threadfence();  // the other arrivers' partials before the ready words
+    word = kReadyMerge | (static_cast<unsigned long long>(t.gtile - t.tile) << 2) |
+           (static_cast<unsigned long long>(ntot) << 32);
+  }
+  st_ready4(p.ws_ready + 4 * static_cast<int64_t>(t.b), word);
+}
+
 // ---------------------------------------------------------------------------
 // Block-wide plan: total tiles, this CTA's tile range and its first sequence.
 // ---------------------------------------------------------------------------
@@ -361,10 +446,6 @@ __device__ void balanced_plan(const DecodeParams& p, DecodeCtrl& c, const int* l
       c.b_start = tid;
       c.off_start = static_cast<int>(t0 - excl);
     }
-    if (blockIdx.x == 0) {  // the combine kernel's view of the plan
-      if (tid < p.batch) p.ws_prefix[tid] = static_cast<int>(excl);
-      if (tid == 0) p.ws_prefix[p.batch] = static_cast<int>(total);
-    }
     located = true;
   } else {
     for (int base = 0; base < p.batch; base += kDecodeThreads) {
@@ -384,7 +465,7 @@ __device__ void balanced_plan(const DecodeParams& p, DecodeCtrl& c, const int* l
   }
   if (!located) {
     long long run = 0;
-    for (int base = 0; base < p.batch && (run <= t0 || blockIdx.x == 0); base += kDecodeThreads) {
+    for (int base = 0; base < p.batch && run <= t0; base += kDecodeThreads) {
       const int b = base + tid;
       const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
       int chunk;
@@ -394,10 +475,8 @@ __device__ void balanced_plan(const DecodeParams& p, DecodeCtrl& c, const int* l
         c.b_start = b;
         c.off_start = static_cast<int>(t0 - excl);
       }
-      if (blockIdx.x == 0 && b < p.batch) p.ws_prefix[b] = static_cast<int>(excl);
       run += chunk;
     }
-    if (blockIdx.x == 0 && tid == 0) p.ws_prefix[p.batch] = static_cast<int>(total);
   }
   __syncthreads();
 }
@@ -555,7 +634,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #ifdef MFA_TRACE
   const unsigned long long gt_start = global_timer_ns();
 #endif
-  griddep_launch_dependents();
 
   // ---- setup (independent of the previous kernel's results) ----------------
   if (tid == 0) {
@@ -580,6 +658,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     mbar_init(&c.q_conv, 1);
     mbar_init(&c.drain, 1);
     c.abort_flag = 0;
+    c.seg_arrivals = 0;
     c.b_start = 0;
     c.off_start = 0;
     fence_mbar_init();
@@ -596,6 +675,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   // ---- plan (reads seq_lens: after the previous kernel has completed) -----
   griddep_wait();
+  // The combine kernel may start from here on: it waits for each sequence's
+  // partials on the synchronisation words, which the previous call (complete
+  // now) left at zero.
+  griddep_launch_dependents();
 #ifdef MFA_TRACE
   const int gt_call = blockIdx.x < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[blockIdx.x]) : -1;
   if (tid == 0) {
@@ -688,7 +771,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const int page = is_k ? pgk : pgv;
         const int nbox = is_k ? nbk : nbv;
         const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+#ifdef MFA_TRACE
         const int kind = is_k ? 0 : 1;
+#endif
         const int t0 = t.tile * kTile;
         const uint32_t bytes =
             four_d ? kSlotBytes : static_cast<uint32_t>(nbox * rows * 128 * kBoxes);
@@ -770,13 +855,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         // head dims 0-127 first, so their ring slot is released half-way
 #pragma unroll
         for (int s = 0; s < kTile / 16; ++s)
-          mma_f16_ss(tmem + kColOlo, sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
+          mma_f16_ss(tmem + o_cols(t.seg) + kColOlo, sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
                      sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
                      (t.seg_first && s == 0) ? 0u : 1u);
         mma_commit(&c.slot_empty[lo % kSlots]);
 #pragma unroll
         for (int s = 0; s < kTile / 16; ++s)
-          mma_f16_ss(tmem + kColOhi, sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
+          mma_f16_ss(tmem + o_cols(t.seg) + kColOhi, sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
                      sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
                      (t.seg_first && s == 0) ? 0u : 1u);
         mma_commit(&c.slot_empty[hi % kSlots]);
@@ -889,6 +974,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         ++g;
       }
       if (ok && g >= 1) ok = convert_item() && convert_item();    // V of the last tile
+    } else {
+      // ======================= segment publisher (bf16 cache) ==============
+      // After the softmax warps have written a segment's output or partial,
+      // makes it visible device-wide and tells the combine kernel.
+      TileStream ns;
+      ns.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+      TileInfo t;
+      unsigned k = 0;
+      while (ns.next(t)) {
+        if (!t.seg_last) continue;
+        ++k;
+        if (!__all_sync(0xffffffffu, wait_count(&c.seg_arrivals, 4u * kWG * k, abort_flag))) break;
+        if (lane == 0) publish_segment(p, t, c.ntot, 1u);
+        __syncwarp();
+      }
     }
   } else if (warp >= 4) {
     // ======================= softmax + epilogue =============================
@@ -908,6 +1008,44 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const float sl2 = p.score_log2;
     float* mv = c.mv[wg][sub];
     float* cv = c.cv[wg][sub];
+    float* ev = c.ev[wg][sub];  // output scale of the pending segment, per head
+
+    // Reads a finished segment's O (its own TMEM pair) and writes this warp's
+    // share: the normalised output, or the partial of a split sequence. Then
+    // hands the segment to its publisher: warp 3 for a bf16 cache (idle
+    // there), so these warps go on without waiting for their stores to drain;
+    // with an FP8 cache (warp 3 converts) every warp arrives itself.
+    TileInfo pend;
+    bool have_pending = false;
+    uint32_t pend_g = 0;  // tile counter of the pending segment's last tile
+    auto write_segment = [&](const TileInfo& pt) {
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const int d = half * 128 + row;
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + o_cols(pt.seg) + (half ? kColOhi : kColOlo) + hbase, r);
+        tmem_wait_ld();
+        if (pt.slot >= 0) {
+          // partial layout [slot][head][d]: a warp writes 128 contiguous bytes per head
+          float* dst = p.ws_o + static_cast<int64_t>(pt.slot) * kPartialFloats +
+                       static_cast<int64_t>(hbase) * kDim + d;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[j * kDim] = __uint_as_float(r[j]) * ev[j];
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            store_out(p, pt.b, hbase + j, d, __uint_as_float(r[j]) * ev[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (!kFp8) {
+        if (lane == 0) smem_add_release(&c.seg_arrivals, 1u);
+      } else if (lane == 0 && (pt.slot >= 0 || warp == 4)) {
+        publish_segment(p, pt, c.ntot, 4u * kWG);
+      }
+      if (warp == 4 && lane == 0) MFA_TR(8, pend_g);
+    };
 
     while (ts.next(t)) {
       if (t.seg_first) m_run = -INFINITY;  // (l_part is zero at every segment start)
@@ -991,7 +1129,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         for (int q4 = 0; q4 < 4; ++q4) {  // (O_lo, O_hi) x two 16-column chunks
           uint32_t r[16];
           const int cb = (q4 & 1) * 16;
-          const uint32_t a = tmem + lane_addr + ((q4 >> 1) ? kColOhi : kColOlo) + hbase + cb;
+          const uint32_t a =
+              tmem + lane_addr + o_cols(t.seg) + ((q4 >> 1) ? kColOhi : kColOlo) + hbase + cb;
           tmem_ld16(a, r);
           tmem_wait_ld();
 #pragma unroll
@@ -1028,7 +1167,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (lane == 0) mbar_arrive(&c.p_full);
       if (warp == 4 && lane == 0) MFA_TR(7, g);
 
-      // ---- epilogue at the end of a segment -------------------------------
+      // ---- output of the previous segment, deferred to here ---------------
+      // Its last PV completed before this tile's P went out (the o_full wait
+      // above) and the MMA now accumulates into the other O pair, so the
+      // read-out overlaps this tile's PV and the next tile's QK.
+      if (have_pending) {
+        write_segment(pend);
+        have_pending = false;
+      }
+
+      // ---- end of a segment: row sums and log-sum-exp ---------------------
       if (t.seg_last) {
         {
           float v[kWGHeads];
@@ -1045,7 +1193,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 #pragma unroll
         for (int h = 0; h < kWGHeads; ++h) l_part[h] = 0.f;
         const float lse = (m_run + lg2_approx(l)) * kLn2;  // head hbase + lane
-        cv[lane] = p.out_scale / l;
+        ev[lane] = p.out_scale / l;
         if (sub == 0) {
           if (t.slot >= 0)
             p.ws_lse[static_cast<int64_t>(t.slot) * kHeads + hbase + lane] = lse;
@@ -1053,32 +1201,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             p.lse_out[t.b * p.lse_sb + hbase + lane] = lse;
         }
         __syncwarp();
-        if (!warp_wait(&c.o_full, par(g), abort_flag)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          const int d = half * 128 + row;
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + (half ? kColOhi : kColOlo) + hbase, r);
-          tmem_wait_ld();
-          if (t.slot >= 0) {
-            // partial layout [slot][head][d]: a warp writes 128 contiguous bytes per head
-            float* dst = p.ws_o + static_cast<int64_t>(t.slot) * kPartialFloats +
-                         static_cast<int64_t>(hbase) * kDim + d;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) dst[j * kDim] = __uint_as_float(r[j]) * cv[j];
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              store_out(p, t.b, hbase + j, d, __uint_as_float(r[j]) * cv[j]);
-          }
-        }
-        tc_fence_before();
-        if (warp == 4 && lane == 0) MFA_TR(8, g);
         ++nseg;
-
+        pend = t;
+        pend_g = g;
+        have_pending = true;
       }
       ++g;
+    }
+    // the CTA's last segment: after its last PV
+    if (have_pending && !*abort_flag && warp_wait(&c.o_full, par(g - 1), abort_flag)) {
+      tc_fence_after();
+      write_segment(pend);
     }
   }
 
@@ -1102,16 +1235,81 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 //   lse* = max_s lse_s,  w_s = exp(lse_s - lse*),
 //   out = sum_s w_s O_s / sum_s w_s,   lse = lse* + log(sum_s w_s)
 // over the sequence's partials in plan order.
+//
+// The kernel starts while the attention kernel still runs (on SMs it has
+// left) and merges each sequence as soon as its ready word says its partials
+// are written, so merges overlap the attention kernel's last tiles. It waits
+// for the attention grid to complete only at its end, so a call is over when
+// this kernel is.
 // ===========================================================================
 constexpr int kCombineHeads = 16;  // heads per CTA
+constexpr int kCombineDims = 16;   // head-dim elements per thread (kDim / 16 threads per head)
+constexpr int kCombineBatch = 4;   // partials loaded per round trip
+
+// Waits (bounded) until *w is non-zero; returns it, or 0 after the wait limit.
+__device__ unsigned long long wait_ready(const unsigned long long* w) {
+  unsigned long long v = ld_acquire_u64(w);
+  if (v != 0) return v;
+  const uint64_t t0 = global_timer_ns();
+  while ((v = ld_acquire_u64(w)) == 0) {
+    __nanosleep(128);
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      record_error(6 /* MFA_ERR_TIMEOUT */);
+      return 0;
+    }
+  }
+  return v;
+}
+
+// 16 consecutive output elements of (b, h) from d0 (16-byte vector stores
+// when the address allows).
+__device__ __forceinline__ void store_out16(const DecodeParams& p, int b, int h, int d0,
+                                            const float* v) {
+  const int64_t off = static_cast<int64_t>(b) * p.out_sb + static_cast<int64_t>(h) * p.out_sh + d0;
+  if (p.out_f32) {
+    float* dst = static_cast<float*>(p.out) + off;
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+      for (int j = 0; j < kCombineDims / 4; ++j)
+        reinterpret_cast<float4*>(dst)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kCombineDims; ++j) dst[j] = v[j];
+    }
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + off;
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+      for (int j = 0; j < kCombineDims / 8; ++j)
+        reinterpret_cast<uint4*>(dst)[j] =
+            make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                       pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < kCombineDims; ++j) dst[j] = __float2bfloat16_rn(v[j]);
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams p) {
 #ifdef MFA_TRACE
   const unsigned long long gt_start = global_timer_ns();
   const int cta_lin = blockIdx.x * gridDim.y + blockIdx.y;
 #endif
-  griddep_wait();  // partials, prefix and lengths come from the attention kernel
   griddep_launch_dependents();
+  const int b = blockIdx.x;
+  const int q = blockIdx.y;
+  const int h = q * kCombineHeads + (threadIdx.x >> 4);  // this thread's head
+  const int d0 = (threadIdx.x & 15) * kCombineDims;       // and its 16 dims
+  // the lengths are an input of the call: complete before the attention
+  // kernel passed its own dependency wait, which precedes this kernel's start
+  const int nt = tiles_of(valid_len(p, b));
+
+  __shared__ unsigned long long s_word;
+  unsigned long long* ready = p.ws_ready + 4 * static_cast<int64_t>(b) + q;
+  if (nt > 0 && threadIdx.x == 0) s_word = wait_ready(ready);
+  __syncthreads();
+  const unsigned long long word = nt > 0 ? s_word : 0;
 #ifdef MFA_TRACE
   const int gt_call = cta_lin < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[kGtCtas + cta_lin]) : -1;
   if (threadIdx.x == 0) {
@@ -1130,74 +1328,78 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
     }
   } gt_end{gt_call, cta_lin};
 #endif
-  const int b = blockIdx.x;
-  const int h0 = blockIdx.y * kCombineHeads;
-  const int d = threadIdx.x;
 
-  SplitList sl;
-  int nt;
-  if (p.num_splits == 0) {
-    const long long S = __ldcg(p.ws_prefix + b);
-    nt = static_cast<int>(__ldcg(p.ws_prefix + b + 1) - S);
-    const long long N = __ldcg(p.ws_prefix + p.batch);
-    if (nt > 0) sl.init_balanced(S, nt, N, p.grid);
-  } else {
-    nt = tiles_of(valid_len(p, b));
-    if (nt > 0) sl.init_fixed(b, nt, p.num_splits);
-  }
+  float v[kCombineDims];
   if (nt == 0) {  // empty sequence: zeros, lse = -inf
 #pragma unroll
-    for (int j = 0; j < kCombineHeads; ++j) store_out(p, b, h0 + j, d, 0.f);
-    if (p.lse_out && d < kCombineHeads) p.lse_out[b * p.lse_sb + h0 + d] = -INFINITY;
-    return;
-  }
-  if (sl.nonempty() <= 1) return;  // written directly by the attention kernel
+    for (int j = 0; j < kCombineDims; ++j) v[j] = 0.f;
+    store_out16(p, b, h, d0, v);
+    if (p.lse_out && d0 == 0) p.lse_out[b * p.lse_sb + h] = -INFINITY;
+  } else if ((word & 3) == kReadyMerge) {
+    SplitList sl;
+    if (p.num_splits == 0)
+      sl.init_balanced(static_cast<long long>((word & 0xffffffffull) >> 2), nt,
+                       static_cast<long long>(word >> 32), p.grid);
+    else
+      sl.init_fixed(b, nt, p.num_splits);
 
-  // online merge over the partials in plan order, two slots per step:
-  // running max m, running weight sum l and running weighted sum acc per head
-  float m[kCombineHeads], l[kCombineHeads], acc[kCombineHeads];
+    // online merge in plan order, up to four partials per step: running max
+    // m, running weight sum l and running weighted sums acc of this head
+    float m = -INFINITY, l = 0.f;
 #pragma unroll
-  for (int j = 0; j < kCombineHeads; ++j) {
-    m[j] = -INFINITY;
-    l[j] = 0.f;
-    acc[j] = 0.f;
-  }
-  for (int i = 0; i < sl.count; i += 2) {
-    const int sa = sl.slot(i);
-    const int sb = i + 1 < sl.count ? sl.slot(i + 1) : -1;
-    if (sa < 0 && sb < 0) continue;
-    float la[kCombineHeads], lb[kCombineHeads], va[kCombineHeads], vb[kCombineHeads];
-    const float* oa = p.ws_o + static_cast<int64_t>(sa < 0 ? 0 : sa) * kPartialFloats +
-                      static_cast<int64_t>(h0) * kDim + d;
-    const float* ob = p.ws_o + static_cast<int64_t>(sb < 0 ? 0 : sb) * kPartialFloats +
-                      static_cast<int64_t>(h0) * kDim + d;
-    const float* ea = p.ws_lse + static_cast<int64_t>(sa < 0 ? 0 : sa) * kHeads + h0;
-    const float* eb = p.ws_lse + static_cast<int64_t>(sb < 0 ? 0 : sb) * kHeads + h0;
+    for (int j = 0; j < kCombineDims; ++j) v[j] = 0.f;
+    for (int i = 0; i < sl.count; i += kCombineBatch) {
+      int slot[kCombineBatch];
+      bool any = false;
 #pragma unroll
-    for (int j = 0; j < kCombineHeads; ++j) {
-      la[j] = sa >= 0 ? __ldcg(ea + j) : -INFINITY;
-      lb[j] = sb >= 0 ? __ldcg(eb + j) : -INFINITY;
-      va[j] = sa >= 0 ? __ldcg(oa + j * kDim) : 0.f;
-      vb[j] = sb >= 0 ? __ldcg(ob + j * kDim) : 0.f;
+      for (int k = 0; k < kCombineBatch; ++k) {
+        slot[k] = i + k < sl.count ? sl.slot(i + k) : -1;
+        any |= slot[k] >= 0;
+      }
+      if (!any) continue;  // empty units of a fixed split
+      float e[kCombineBatch];
+      float4 o[kCombineBatch][kCombineDims / 4];
+#pragma unroll
+      for (int k = 0; k < kCombineBatch; ++k) {
+        const int sk = slot[k] < 0 ? 0 : slot[k];
+        const float4* src = reinterpret_cast<const float4*>(
+            p.ws_o + static_cast<int64_t>(sk) * kPartialFloats + static_cast<int64_t>(h) * kDim + d0);
+        e[k] = slot[k] >= 0 ? __ldcg(p.ws_lse + static_cast<int64_t>(sk) * kHeads + h) : -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kCombineDims / 4; ++j)
+          o[k][j] = slot[k] >= 0 ? __ldcg(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float mn = m;
+#pragma unroll
+      for (int k = 0; k < kCombineBatch; ++k) mn = fmaxf(mn, e[k]);  // finite: one slot is valid
+      const float c = ex2_approx((m - mn) * kLog2e);
+      l *= c;
+#pragma unroll
+      for (int j = 0; j < kCombineDims; ++j) v[j] *= c;
+#pragma unroll
+      for (int k = 0; k < kCombineBatch; ++k) {
+        const float w = ex2_approx((e[k] - mn) * kLog2e);
+        l += w;
+#pragma unroll
+        for (int j = 0; j < kCombineDims / 4; ++j) {
+          v[4 * j] += w * o[k][j].x;
+          v[4 * j + 1] += w * o[k][j].y;
+          v[4 * j + 2] += w * o[k][j].z;
+          v[4 * j + 3] += w * o[k][j].w;
+        }
+      }
+      m = mn;
     }
+    const float inv = 1.f / l;
 #pragma unroll
-    for (int j = 0; j < kCombineHeads; ++j) {
-      const float mn = fmaxf(m[j], fmaxf(la[j], lb[j]));  // finite: one slot is valid
-      const float c = ex2_approx((m[j] - mn) * kLog2e);
-      const float wa = ex2_approx((la[j] - mn) * kLog2e);
-      const float wb = ex2_approx((lb[j] - mn) * kLog2e);
-      l[j] = l[j] * c + wa + wb;
-      acc[j] = acc[j] * c + wa * va[j] + wb * vb[j];
-      m[j] = mn;
-    }
+    for (int j = 0; j < kCombineDims; ++j) v[j] *= inv;
+    store_out16(p, b, h, d0, v);
+    if (p.lse_out && d0 == 0) p.lse_out[b * p.lse_sb + h] = m + lg2_approx(l) * kLn2;
   }
-#pragma unroll
-  for (int j = 0; j < kCombineHeads; ++j) store_out(p, b, h0 + j, d, acc[j] / l[j]);
-  if (p.lse_out && d == 0) {
-#pragma unroll
-    for (int j = 0; j < kCombineHeads; ++j)
-      p.lse_out[b * p.lse_sb + h0 + j] = m[j] + lg2_approx(l[j]) * kLn2;
-  }
+  // back to zero for the next call, which sets it only after this kernel
+  // has completed
+  if (nt > 0 && threadIdx.x == 0 && word != 0) *ready = 0;
+  griddep_wait();
 }
 
 // ===========================================================================

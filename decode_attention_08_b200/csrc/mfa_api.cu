@@ -173,18 +173,53 @@ int cached_workspace(CachedWs* table, size_t need, bool zero, void** out) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Decode workspace: the plan's per-sequence tile prefix, then the partial
-// outputs of split sequences and their log-sum-exp values.
+// The batch size each recently used decode workspace last served (a small
+// round-robin table): the synchronisation words of a workspace not in it, or
+// last used with another batch size, may not be at zero where this call
+// looks for them.
+struct WsMemo {
+  const void* ptr = nullptr;
+  int batch = 0;
+};
+constexpr int kWsMemo = 64;
+WsMemo g_ws_memo[kWsMemo];
+int g_ws_memo_next = 0;
+
+void forget_workspaces() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (WsMemo& m : g_ws_memo) m = WsMemo{};
+}
+
+bool sync_words_stale(const void* ws, int batch) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (WsMemo& m : g_ws_memo) {
+    if (m.ptr == ws) {
+      const bool stale = m.batch != batch;
+      m.batch = batch;
+      return stale;
+    }
+  }
+  g_ws_memo[g_ws_memo_next] = {ws, batch};
+  g_ws_memo_next = (g_ws_memo_next + 1) % kWsMemo;
+  return true;
+}
+
+// Decode workspace: the per-sequence synchronisation words between the
+// attention and the combine kernel (an arrival counter, four ready words),
+// then the partial outputs of split sequences and their log-sum-exp values.
 struct DecodeWsLayout {
-  size_t prefix_off, o_off, lse_off, total;
+  size_t arrive_off, ready_off, sync_bytes, o_off, lse_off, total;
   int slots;
 };
 
 DecodeWsLayout decode_ws_layout(int batch, int num_splits, int grid) {
   DecodeWsLayout l;
+  const size_t B = static_cast<size_t>(batch);
   l.slots = num_splits == 0 ? 2 * grid : batch * num_splits;
-  l.prefix_off = 0;
-  l.o_off = align256(static_cast<size_t>(batch + 1) * sizeof(int));
+  l.arrive_off = 0;
+  l.ready_off = (B * sizeof(unsigned) + 15) & ~static_cast<size_t>(15);
+  l.sync_bytes = align256(l.ready_off + B * 4 * sizeof(unsigned long long));
+  l.o_off = l.sync_bytes;
   l.lse_off = align256(l.o_off + static_cast<size_t>(l.slots) * kPartialFloats * sizeof(float));
   l.total = align256(l.lse_off + static_cast<size_t>(l.slots) * kHeads * sizeof(float));
   return l;
@@ -414,8 +449,17 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
   p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
-  p.ws_prefix = reinterpret_cast<int*>(ws + wl.prefix_off);
+  p.ws_arrive = reinterpret_cast<unsigned*>(ws + wl.arrive_off);
+  p.ws_ready = reinterpret_cast<unsigned long long*>(ws + wl.ready_off);
 
+  // Every call leaves the synchronisation words it used at zero; they sit at
+  // batch-dependent offsets, so a workspace seen for the first time or with
+  // another batch size has them cleared first.
+  if (sync_words_stale(workspace, static_cast<int>(B))) {
+    const cudaError_t e =
+        cudaMemsetAsync(workspace, 0, wl.sync_bytes, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   const cudaError_t err =
       launch_decode(paged, fp8, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? MFA_OK : cuda_fail(err);
@@ -446,7 +490,7 @@ int mfa_decode_attention(const mfa_tensor* q, const mfa_tensor* k_cache,
   const size_t need = mfa_decode_workspace_size(static_cast<int>(q->shape[0]), 0);
   if (need == 0) return MFA_ERR_CUDA;
   void* ws = nullptr;
-  const int rc = cached_workspace(g_ws_decode, need, false, &ws);
+  const int rc = cached_workspace(g_ws_decode, need, true, &ws);
   if (rc != MFA_OK) return rc;
   return mfa_decode_attention_ex(q, k_cache, v_cache, page_table, seq_lens, out, softmax_scale,
                                  kv_dtype, 1.f, 1.f, 0, nullptr, ws, need, stream);
@@ -565,6 +609,9 @@ int mfa_read_status(mfa_stream_t stream, int reset, int* status_out) {
     e = cudaMemcpyToSymbol(g_mfa_status, &zero, sizeof zero);
     if (e != cudaSuccess) return cuda_fail(e);
   }
+  // a failed call (an aborted wait) may leave synchronisation words set:
+  // clear every workspace's words on its next use
+  if (v != 0) forget_workspaces();
   *status_out = v;
   return MFA_OK;
 }

@@ -19,7 +19,10 @@ constexpr int kSlotBytes = 128 * 128 * 2;  // one tensor, 128 tokens x 128 dims,
 constexpr int kQBytes = kHeads * kDim * 2;
 constexpr int kPBytes = kTile * kHeads * 2;
 constexpr int kDecodeThreads = 384;        // 12 warps: 4 service warps + 2 softmax warpgroups
-constexpr int kTmemCols = 256;             // S0 | S1 | O_lo | O_hi, 64 columns each
+// S0 | S1 | O_lo | O_hi for even segments | (unused) | O_lo | O_hi for odd
+// segments, 64 columns each: a segment's output is read out while the next
+// segment accumulates into the other pair
+constexpr int kTmemCols = 512;
 
 // One partial (split) result: O [64 heads][256 d] f32, normalised over its range.
 constexpr size_t kPartialFloats = static_cast<size_t>(kHeads) * kDim;
@@ -45,8 +48,17 @@ struct DecodeParams {
   int64_t lse_sb;
   float* ws_o;             // [slots][64 heads][256 d] normalised partial outputs
   float* ws_lse;           // [slots][64] their log-sum-exp (natural log)
-  int* ws_prefix;          // [B + 1] first global tile of each sequence (balanced plan)
+  // synchronisation words between the attention and the combine kernel; zero
+  // between calls (each call returns them to zero)
+  unsigned* ws_arrive;     // [B] segment arrivals of a split sequence
+  // [B][4] one word per combine CTA of the sequence: bits 0-1 the state (0
+  // pending, kReadyNone, kReadyMerge), bits 2-31 the sequence's first global
+  // tile, bits 32-63 the batch's total tiles (balanced plan)
+  unsigned long long* ws_ready;
 };
+
+constexpr unsigned kReadyNone = 1;   // the attention kernel wrote the sequence's output itself
+constexpr unsigned kReadyMerge = 2;  // every partial of the sequence is written
 
 struct QprojParams {
   int batch;

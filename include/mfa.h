@@ -110,8 +110,17 @@ int mfa_decode_attention(const mfa_tensor* q, const mfa_tensor* k_cache,
  *                    scores (-inf for empty sequences).
  *  workspace         device memory of at least
  *                    mfa_decode_workspace_size(B, num_splits) bytes, 256-byte
- *                    aligned. Contents need no initialisation. Calls that
- *                    overlap on the GPU must not share a workspace.
+ *                    aligned. Its first bytes hold synchronisation words
+ *                    between the call's two kernels, which every call leaves
+ *                    at zero. The library clears them itself (one
+ *                    cudaMemsetAsync on the call's stream) the first time it
+ *                    sees a workspace address and whenever the batch size
+ *                    changes, and for every workspace after mfa_read_status
+ *                    has reported a non-zero status (a call that gave up a
+ *                    wait may leave them set). Between calls the caller must
+ *                    not write to the workspace. Calls that overlap on the GPU
+ *                    must not share a workspace, and a CUDA graph that
+ *                    captured a call needs its workspace to itself.
  * Splitting never changes which cached rows contribute; the split plan depends
  * only on seq_lens, num_splits and the SM count, never on the cache layout, so a
  * paged and a contiguous cache holding the same rows give bit-identical results.
