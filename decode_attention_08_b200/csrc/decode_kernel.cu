@@ -84,7 +84,7 @@ struct __align__(16) DecodeCtrl {
   uint64_t slot_full[kSlots], slot_empty[kSlots];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, o_full;
-  uint64_t conv_full[kSlots], q_conv;  // FP8 cache: ring slot / q expanded to f16
+  uint64_t q_conv;  // FP8 cache: q converted to its E4M3 pair
   uint64_t red_full[kWG][2], l_full[kWG];
   uint64_t drain;
   long long t0;    // first global tile of this CTA (balanced plan)
@@ -92,6 +92,8 @@ struct __align__(16) DecodeCtrl {
   uint32_t tmem_base;
   int abort_flag;
   unsigned seg_arrivals;  // bf16 cache: softmax-warp arrivals at segment ends (never wraps)
+  unsigned q_ready;       // FP8 cache: segments whose q is converted (never wraps)
+  float qinv[4];          // FP8 cache: score scale 1/s of segment k at [k & 3]
   int b_start, off_start, tiles;
   int scan_warp[kDecodeThreads / 32];
   int lens[kDecodeThreads];  // validated seq_lens when batch <= kDecodeThreads
@@ -114,12 +116,20 @@ constexpr int kSmemBytes = kSmemCtrl + static_cast<int>(sizeof(DecodeCtrl)) + 10
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // TMEM column map.
-constexpr uint32_t kColS = 0;      // two 64-column score buffers
+constexpr uint32_t kColS = 0;      // score buffers: bf16 cols 0-63 | 64-127; FP8 0-127 | 256-383
 constexpr uint32_t kColOlo = 128;  // O^T rows 0..127
 constexpr uint32_t kColOhi = 192;  // O^T rows 128..255
 constexpr uint32_t kColObuf = 256; // column offset of the odd segments' O pair
 
 __device__ __forceinline__ uint32_t o_cols(int seg) { return (seg & 1) ? kColObuf : 0u; }
+
+// Score buffer of tile g. bf16: 64 columns (heads). FP8: 128 columns, K.q_hi
+// in 0-63 and K.q_lo in 64-127 (one N = 128 product per step reads each K
+// step once for both parts).
+template <bool kFp8>
+__device__ __forceinline__ uint32_t s_cols(uint32_t g) {
+  return kColS + (g & 1) * (kFp8 ? 256u : 64u);
+}
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -514,11 +524,17 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[kWGHeads], int lane
   return v[0];
 }
 
-// Index, in producer order, of the first (lo) ring item holding V of the CTA's
-// j-th tile: items go K0 | K1 V0 | K2 V1 | ... | K(T-1) V(T-2) | V(T-1), two
-// items (lo/hi head-dim halves) per tensor and tile.
+// Ring items per tensor and tile: bf16 K or V tiles take two 32 KB slots (head
+// dims 0-127, 128-255); an E4M3 tile fits one slot (its two 16 KB halves).
+template <bool kFp8>
+constexpr uint32_t kItemsPerTensor = kFp8 ? 1u : 2u;
+
+// Index, in producer order, of the first ring item holding V of the CTA's j-th
+// tile: items go K0 | K1 V0 | K2 V1 | ... | K(T-1) V(T-2) | V(T-1).
+template <bool kFp8>
 __device__ __forceinline__ uint32_t v_item(uint32_t j, bool cta_last) {
-  return cta_last ? 4u * j + 2u : 4u * j + 4u;
+  constexpr uint32_t n = kItemsPerTensor<kFp8>;
+  return cta_last ? 2u * n * j + n : 2u * n * j + 2u * n;
 }
 
 // Page ids of 32 consecutive logical pages of one sequence, one per lane of the
@@ -550,62 +566,73 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
-// two E4M3 codes (low byte = first element) -> f16x2, exact
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  uint32_t out;
-  const uint16_t in = static_cast<uint16_t>(two_codes);
-  asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
-      : "=r"(out)
-      : "h"(in));
-  return out;
+// FP8 cache, per segment: q (bf16, 64 heads x 256 dims, as TMA wrote it: four
+// 8 KB regions of 64 dims, 128-byte rows with the 128-byte swizzle) becomes two
+// E4M3 operands whose sum is q * s exactly (s a power of two putting max|q*s|
+// in [128, 256); bf16's 8 significant bits split into two 4-bit parts):
+// dims half c (0, 1) -> hi at 16 KB * c, lo at 16 KB * c + 8 KB, each 64 rows
+// of 128 dims (128-byte rows, 128-byte swizzle). Returns 1 / s.
+
+// max |q| over the tile (all lanes get it)
+__device__ __forceinline__ float q_max_abs(uint32_t base, int lane) {
+  uint32_t m = 0;
+#pragma unroll 8
+  for (int i = lane; i < kQBytes / 16; i += 32) {
+    const uint4 v = ld_shared_v4(base + i * 16);
+    m = __vmaxu2(m, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                             __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = __vmaxu2(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const uint32_t top = (m >> 16) > (m & 0xFFFFu) ? (m >> 16) : (m & 0xFFFFu);
+  return __uint_as_float(top << 16);
 }
 
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
-  const __half2 h = __floats2half2_rn(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// FP8 cache: expand one ring slot in place. TMA wrote an E4M3 half-tile of 128
-// token rows x 128 head dims (128-byte rows, 128-byte swizzle) into the slot's
-// first 16 KB; it becomes the f16 half-tile the MMA reads: two 16 KB regions
-// (dims 0-63, 64-127) of 128-byte swizzled rows. Each lane owns whole rows: it
-// reads its row completely before writing, and region 0's row r sits exactly on
-// input row r, so no row is overwritten before it has been read.
-__device__ __forceinline__ void expand_fp8_halftile(uint32_t base, int lane) {
+__device__ __forceinline__ float q_to_e4m3(uint32_t base, int lane) {
+  // s = 2^(7 - E) with max|q| in [2^E, 2^(E+1)); the exponent field is clamped
+  // so that s and 1/s stay normal floats (an all-zero q takes any scale)
+  int ebits = static_cast<int>((__float_as_uint(q_max_abs(base, lane)) >> 23) & 0xFF);
+  ebits = ebits < 8 ? 8 : (ebits > 253 ? 253 : ebits);
+  const float s = __uint_as_float(static_cast<uint32_t>(261 - ebits) << 23);
+  const float inv_s = __uint_as_float(static_cast<uint32_t>(ebits - 7) << 23);
 #pragma unroll 1
-  for (int row = lane; row < kTile; row += 32) {
-    const uint32_t in = base + row * 128;
-    const int sw = row & 7;
-    uint4 v[8];
+  for (int h = lane; h < kHeads; h += 32) {
+    const int sw = h & 7;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      // the whole row of this head and dims half first: the outputs land on it
+      uint4 in[16];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) v[c] = ld_shared_v4(in + ((c ^ sw) << 4));
+      for (int k = 0; k < 2; ++k)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {  // input chunk c = dims 16c..16c+15
-      const uint32_t dst = base + (c >> 2) * (kSlotBytes / 2) + row * 128;
-      const int c2 = (c & 3) * 2;
-      st_shared_v4(dst + ((c2 ^ sw) << 4), e4m3x2_to_f16x2(v[c].x),
-                   e4m3x2_to_f16x2(v[c].x >> 16), e4m3x2_to_f16x2(v[c].y),
-                   e4m3x2_to_f16x2(v[c].y >> 16));
-      st_shared_v4(dst + (((c2 + 1) ^ sw) << 4), e4m3x2_to_f16x2(v[c].z),
-                   e4m3x2_to_f16x2(v[c].z >> 16), e4m3x2_to_f16x2(v[c].w),
-                   e4m3x2_to_f16x2(v[c].w >> 16));
+        for (int j = 0; j < 8; ++j)
+          in[8 * k + j] = ld_shared_v4(base + (2 * c + k) * 8192 + h * 128 + ((j ^ sw) << 4));
+      const uint32_t hi_row = base + c * 16384 + h * 128;
+      const uint32_t lo_row = hi_row + 8192;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {  // output chunk m: dims 16m..16m+15 of the half
+        uint32_t w[8];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const uint4 v = in[2 * m + u];
+          const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            // four bf16 -> two hi/lo pairs
+            const uint32_t p0 = split_e4m3x2(__uint_as_float(wd[e] << 16) * s,
+                                             __uint_as_float(wd[e] & 0xFFFF0000u) * s);
+            const uint32_t p1 = split_e4m3x2(__uint_as_float(wd[e + 1] << 16) * s,
+                                             __uint_as_float(wd[e + 1] & 0xFFFF0000u) * s);
+            w[4 * u + e / 2] = (p0 & 0xFFFFu) | (p1 << 16);          // hi bytes
+            w[4 * u + 2 + e / 2] = (p0 >> 16) | (p1 & 0xFFFF0000u);  // lo bytes
+          }
+        }
+        st_shared_v4(hi_row + ((m ^ sw) << 4), w[0], w[1], w[4], w[5]);
+        st_shared_v4(lo_row + ((m ^ sw) << 4), w[2], w[3], w[6], w[7]);
+      }
     }
   }
-}
-
-// FP8 cache: q (bf16, 32 KB) to f16 in place, for f16 x f16 MMAs.
-__device__ __forceinline__ void q_to_f16(uint32_t base, int lane) {
-#pragma unroll 4
-  for (int i = lane; i < kQBytes / 16; i += 32) {
-    uint4 v = ld_shared_v4(base + i * 16);
-    st_shared_v4(base + i * 16, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                 bf16x2_to_f16x2(v.w));
-  }
+  return inv_s;
 }
 
 }  // namespace
@@ -654,11 +681,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     mbar_init(&c.p_full, 4 * kWG);
     mbar_init(&c.o_full, 1);
-    for (int i = 0; i < kSlots; ++i) mbar_init(&c.conv_full[i], 1);
     mbar_init(&c.q_conv, 1);
     mbar_init(&c.drain, 1);
     c.abort_flag = 0;
     c.seg_arrivals = 0;
+    c.q_ready = 0;
     c.b_start = 0;
     c.off_start = 0;
     fence_mbar_init();
@@ -726,12 +753,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const int num_pages = p.num_pages;
     const int* page_table = p.page_table;
     const int64_t pt_stride = p.pt_stride;
-    // bf16: two boxes of 64 dims x rows per half (or one 4-D box of both);
-    // FP8: one box of 128 dims into the slot's first half, expanded to f16 by
-    // the converter
-    constexpr int kBoxes = kFp8 ? 1 : 2;
+    // bf16: per item (head dims 0-127 or 128-255) two boxes of 64 dims x rows
+    // (or one 4-D box of both); FP8: one item per tensor, two boxes of 128
+    // dims x rows, one per 16 KB half of the slot
+    constexpr int kBoxes = 2;
     constexpr int kBoxDims = kFp8 ? 128 : 64;
-    const bool four_d = !kFp8 && rshift == 7;  // contiguous bf16, or bf16 pages >= 128
+    const bool four_d = rshift == 7;  // contiguous, or pages of >= 128 tokens
 
     // Sub-pages of a tile (paged caches): lane j < nbox loads sub-page j (a
     // page, or the part of a >= 128-token page under the tile) and holds its
@@ -778,7 +805,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const uint32_t bytes =
             four_d ? kSlotBytes : static_cast<uint32_t>(nbox * rows * 128 * kBoxes);
         bool ok = true;
-        for (int half = 0; half < 2 && ok; ++half) {
+        for (int half = 0; half < static_cast<int>(kItemsPerTensor<kFp8>) && ok; ++half) {
           const uint32_t slot = item % kSlots;
           ok = warp_wait(&c.slot_empty[slot], par(item / kSlots) ^ 1u, abort_flag);
           if (!ok) break;
@@ -795,7 +822,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               // stride 128 B) after the token dimension: the box lands as
               // [chunk][128 tokens][128 B]
               tma_load_4d(dst, map, &c.slot_full[slot], 0, kPaged ? (t0 & (ps - 1)) : t0,
-                          2 * half, outer, policy);
+                          kFp8 ? 0 : 2 * half, outer, policy);
             } else {
               const int tok = t0 + (lane << rshift);
               for (int r = 0; r < kBoxes; ++r)
@@ -828,12 +855,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =====================================
-    // operands: bf16 for a bf16 cache; f16 (exact expansion of E4M3, q and P in
-    // f16) for an FP8 cache
-    constexpr int kAB = kFp8 ? 0 : 1;
-    constexpr uint32_t idesc_qk = idesc_f16(128, 64, kAB, 0, 0);
-    constexpr uint32_t idesc_pv = idesc_f16(128, 64, kAB, 1, 1);
-    uint64_t* operand_ready = kFp8 ? c.conv_full : c.slot_full;
+    // bf16 cache: kind::f16 products of bf16 operands. FP8 cache: kind::f8f6f4
+    // products of E4M3 operands straight from the ring (K, V), with q and P
+    // each given as an exact E4M3 pair hi + lo (two products per step).
+    constexpr uint32_t idesc_qk = idesc_f16(128, kFp8 ? 128 : 64, kFp8 ? 0 : 1, 0, 0);
+    constexpr uint32_t idesc_pv = idesc_f16(128, 64, kFp8 ? 0 : 1, 1, 1);
+    constexpr uint32_t kIPT = kItemsPerTensor<kFp8>;
     const uint32_t q_base = smem_u32(sQ);
     const uint32_t ring_base = smem_u32(sRing);
     const uint32_t p_base = smem_u32(sP);
@@ -841,30 +868,57 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     qs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
     uint32_t item = 0, nq = 0;
     bool ok = true;
+    // waits for the kIPT ring items of the next tensor; returns the first
+    auto take_items = [&](uint32_t& first) -> bool {
+      first = item;
+      item += kIPT;
+      for (uint32_t u = 0; u < kIPT; ++u)
+        if (!warp_wait(&c.slot_full[(first + u) % kSlots], par((first + u) / kSlots), abort_flag))
+          return false;
+      return true;
+    };
 
     auto issue_pv = [&](const TileInfo& t, uint32_t j) -> bool {
       if (!warp_wait(&c.p_full, par(j), abort_flag)) return false;
-      const uint32_t lo = item++, hi = item++;
-      if (!warp_wait(&operand_ready[lo % kSlots], par(lo / kSlots), abort_flag)) return false;
-      if (!warp_wait(&operand_ready[hi % kSlots], par(hi / kSlots), abort_flag)) return false;
+      uint32_t lo;
+      if (!take_items(lo)) return false;
       tc_fence_after();
       if (lane == 0) {
         MFA_TR(3, j);
-        const uint32_t v_lo = ring_base + (lo % kSlots) * kSlotBytes;
-        const uint32_t v_hi = ring_base + (hi % kSlots) * kSlotBytes;
-        // head dims 0-127 first, so their ring slot is released half-way
+        const uint32_t d_o = tmem + o_cols(t.seg);
+        if (kFp8) {
+          // V slot: head dims 0-127 | 128-255, each 128 token rows of 128 B
+          // (MN-major A); P hi | lo: 128 token rows of 64 B (MN-major B)
+          const uint32_t v = ring_base + (lo % kSlots) * kSlotBytes;
 #pragma unroll
-        for (int s = 0; s < kTile / 16; ++s)
-          mma_f16_ss(tmem + o_cols(t.seg) + kColOlo, sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
-                     sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
-                     (t.seg_first && s == 0) ? 0u : 1u);
-        mma_commit(&c.slot_empty[lo % kSlots]);
+          for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int s = 0; s < kTile / 16; ++s)
-          mma_f16_ss(tmem + o_cols(t.seg) + kColOhi, sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
-                     sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
-                     (t.seg_first && s == 0) ? 0u : 1u);
-        mma_commit(&c.slot_empty[hi % kSlots]);
+            for (int kk = 0; kk < kTile / 32; ++kk)
+#pragma unroll
+              for (int part = 0; part < 2; ++part)
+                mma_f8_ss(d_o + (r ? kColOhi : kColOlo),
+                          sw128_desc(v + r * (kSlotBytes / 2) + kk * 4096, kSlotBytes / 2, 1024),
+                          sw64_desc(p_base + part * (kPBytes / 2) + kk * 2048, kPBytes / 2, 512),
+                          idesc_pv, (t.seg_first && kk == 0 && part == 0) ? 0u : 1u);
+          mma_commit(&c.slot_empty[lo % kSlots]);
+        } else {
+          const uint32_t hi = lo + 1;
+          const uint32_t v_lo = ring_base + (lo % kSlots) * kSlotBytes;
+          const uint32_t v_hi = ring_base + (hi % kSlots) * kSlotBytes;
+          // head dims 0-127 first, so their ring slot is released half-way
+#pragma unroll
+          for (int s = 0; s < kTile / 16; ++s)
+            mma_f16_ss(d_o + kColOlo, sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
+                       sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                       (t.seg_first && s == 0) ? 0u : 1u);
+          mma_commit(&c.slot_empty[lo % kSlots]);
+#pragma unroll
+          for (int s = 0; s < kTile / 16; ++s)
+            mma_f16_ss(d_o + kColOhi, sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
+                       sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                       (t.seg_first && s == 0) ? 0u : 1u);
+          mma_commit(&c.slot_empty[hi % kSlots]);
+        }
         mma_commit(&c.o_full);
       }
       __syncwarp();
@@ -880,25 +934,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         if (!ok) break;
       }
       if (g >= 2 && !(ok = warp_wait(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag))) break;
-      const uint32_t lo = item++, hi = item++;
-      if (!(ok = warp_wait(&operand_ready[lo % kSlots], par(lo / kSlots), abort_flag))) break;
-      if (!(ok = warp_wait(&operand_ready[hi % kSlots], par(hi / kSlots), abort_flag))) break;
+      uint32_t lo;
+      if (!(ok = take_items(lo))) break;
       tc_fence_after();
       if (lane == 0) {
         MFA_TR(2, g);
-        const uint32_t k_lo = ring_base + (lo % kSlots) * kSlotBytes;
-        const uint32_t k_hi = ring_base + (hi % kSlots) * kSlotBytes;
-        const uint32_t d_s = tmem + kColS + (g & 1) * 64;
+        const uint32_t d_s = tmem + s_cols<kFp8>(g);
+        if (kFp8) {
+          // K slot: head dims 0-127 | 128-255 (128 token rows of 128 B, K-major);
+          // q: per dims half, the 64 hi rows then the 64 lo rows (128 rows of
+          // 128 B, K-major): one N = 128 operand
+          const uint32_t k = ring_base + (lo % kSlots) * kSlotBytes;
 #pragma unroll
-        for (int s = 0; s < kDim / 16; ++s) {
-          const uint32_t a_addr = (s < 8 ? k_lo : k_hi) + ((s >> 2) & 1) * (kSlotBytes / 2) +
-                                  (s & 3) * 32;
-          const uint32_t b_addr = q_base + (s >> 2) * 8192 + (s & 3) * 32;
-          mma_f16_ss(d_s, sw128_desc(a_addr, 16, 1024), sw128_desc(b_addr, 16, 1024), idesc_qk,
-                     s > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kDim / 32; ++kk) {
+            const uint32_t off = (kk >> 2) * (kSlotBytes / 2) + (kk & 3) * 32;
+            mma_f8_ss(d_s, sw128_desc(k + off, 16, 1024), sw128_desc(q_base + off, 16, 1024),
+                      idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&c.slot_empty[lo % kSlots]);
+        } else {
+          const uint32_t hi = lo + 1;
+          const uint32_t k_lo = ring_base + (lo % kSlots) * kSlotBytes;
+          const uint32_t k_hi = ring_base + (hi % kSlots) * kSlotBytes;
+#pragma unroll
+          for (int s = 0; s < kDim / 16; ++s) {
+            const uint32_t a_addr = (s < 8 ? k_lo : k_hi) + ((s >> 2) & 1) * (kSlotBytes / 2) +
+                                    (s & 3) * 32;
+            const uint32_t b_addr = q_base + (s >> 2) * 8192 + (s & 3) * 32;
+            mma_f16_ss(d_s, sw128_desc(a_addr, 16, 1024), sw128_desc(b_addr, 16, 1024), idesc_qk,
+                       s > 0 ? 1u : 0u);
+          }
+          mma_commit(&c.slot_empty[lo % kSlots]);
+          mma_commit(&c.slot_empty[hi % kSlots]);
         }
-        mma_commit(&c.slot_empty[lo % kSlots]);
-        mma_commit(&c.slot_empty[hi % kSlots]);
         mma_commit(&c.s_full[g & 1]);
         if (cur.seg_last) mma_commit(&c.q_empty);
       }
@@ -945,35 +1013,28 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // Follows the MMA's consumption order: q at each segment start, then K of
     // tile g and V of tile g-1, each half-tile expanded in place to f16.
     if (kFp8) {
+      // ======================= q to E4M3 (FP8 cache) ======================
+      // Per segment, after q has landed: q becomes its exact E4M3 pair (see
+      // q_to_e4m3) in place; the score scale 1/s goes to the softmax warps
+      // through a four-entry ring (this warp runs at most two segments ahead
+      // of them: q of the next segment waits for the current one's last QK).
       TileStream cs;
       cs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
-      uint32_t item = 0, nq = 0, g = 0;
-      auto convert_item = [&]() -> bool {
-        const uint32_t slot = item % kSlots;
-        if (!warp_wait(&c.slot_full[slot], par(item / kSlots), abort_flag)) return false;
-        expand_fp8_halftile(smem_u32(sRing + slot * kSlotBytes), lane);
+      TileInfo t;
+      uint32_t nq = 0;
+      while (cs.next(t)) {
+        if (!t.seg_first) continue;
+        if (!warp_wait(&c.q_full, par(nq), abort_flag)) break;
+        const float inv_s = q_to_e4m3(smem_u32(sQ), lane);
+        if (lane == 0) c.qinv[nq & 3] = inv_s;
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&c.conv_full[slot]);
-        ++item;
-        return true;
-      };
-      TileInfo t;
-      bool ok = true;
-      while (ok && cs.next(t)) {
-        if (t.seg_first) {
-          if (!(ok = warp_wait(&c.q_full, par(nq), abort_flag))) break;
-          q_to_f16(smem_u32(sQ), lane);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&c.q_conv);
-          ++nq;
+        if (lane == 0) {
+          mbar_arrive(&c.q_conv);
+          smem_add_release(&c.q_ready, 1u);
         }
-        ok = convert_item() && convert_item();             // K of tile g
-        if (ok && g >= 1) ok = convert_item() && convert_item();  // V of tile g-1
-        ++g;
+        ++nq;
       }
-      if (ok && g >= 1) ok = convert_item() && convert_item();    // V of the last tile
     } else {
       // ======================= segment publisher (bf16 cache) ==============
       // After the softmax warps have written a segment's output or partial,
@@ -1047,8 +1108,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (warp == 4 && lane == 0) MFA_TR(8, pend_g);
     };
 
+    float sl2_seg = sl2;  // score scale of the current segment
     while (ts.next(t)) {
-      if (t.seg_first) m_run = -INFINITY;  // (l_part is zero at every segment start)
+      if (t.seg_first) {
+        m_run = -INFINITY;  // (l_part is zero at every segment start)
+        if (kFp8) {
+          // q of this segment entered the products as q * s: scale by 1/s
+          if (!__all_sync(0xffffffffu, wait_count(&c.q_ready, t.seg + 1, abort_flag))) break;
+          sl2_seg = sl2 * c.qinv[t.seg & 3];
+        }
+      }
       // ---- scores of this tile (this warpgroup's 32 heads) ---------------
       if (!warp_wait(&c.s_full[g & 1], par(g >> 1), abort_flag)) break;
       if (warp == 4 && lane == 0) MFA_TR(4, g);
@@ -1056,10 +1125,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       float s[kWGHeads];
       {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + kColS + (g & 1) * 64 + hbase, r);
-        tmem_wait_ld();
+        tmem_ld32(tmem + lane_addr + s_cols<kFp8>(g) + hbase, r);
+        if (kFp8) {
+          uint32_t r2[32];
+          tmem_ld32(tmem + lane_addr + s_cols<kFp8>(g) + 64 + hbase, r2);
+          tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]);
+          for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]) + __uint_as_float(r2[h]);
+        } else {
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -1068,7 +1145,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const int valid = min(kTile, t.L - t.tile * kTile);
       const bool row_ok = row < valid;
 #pragma unroll
-      for (int h = 0; h < kWGHeads; ++h) s[h] = row_ok ? s[h] * sl2 : -INFINITY;
+      for (int h = 0; h < kWGHeads; ++h) s[h] = row_ok ? s[h] * sl2_seg : -INFINITY;
 
       // ---- per-head maximum over the tile's 128 rows --------------------
       {
@@ -1116,8 +1193,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           l_part[h + 2] += p2;
           l_part[h + 3] += p3;
         }
-        pk[h / 2] = kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
-        pk[h / 2 + 1] = kFp8 ? pack_f16x2(p2, p3) : pack_bf16x2(p2, p3);
+        if (kFp8) {
+          // E4M3 pairs: hi bytes of heads h..h+3 in pk[h / 4], lo bytes in pk[8 + h / 4]
+          const uint32_t a = split_e4m3x2(p0, p1), b = split_e4m3x2(p2, p3);
+          pk[h / 4] = (a & 0xFFFFu) | (b << 16);
+          pk[8 + h / 4] = (a >> 16) | (b & 0xFFFF0000u);
+        } else {
+          pk[h / 2] = pack_bf16x2(p0, p1);
+          pk[h / 2 + 1] = pack_bf16x2(p2, p3);
+        }
       }
 
       // ---- P buffer and O are free once the previous tile's PV completed --
@@ -1139,7 +1223,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
         tmem_wait_st();
       }
-      {
+      if (kFp8) {
+        // P hi | lo: 128 token rows of 64 heads (64 B, 64-byte swizzle); this
+        // warpgroup's 32 heads are 16-byte chunks 2 wg, 2 wg + 1 of the row
+        const uint32_t rowaddr = smem_u32(sP) + row * 64;
+        const int sw = (row >> 1) & 3;
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch)
+            st_shared_v4(rowaddr + part * (kPBytes / 2) + (((2 * wg + ch) ^ sw) << 4),
+                         pk[8 * part + 4 * ch], pk[8 * part + 4 * ch + 1],
+                         pk[8 * part + 4 * ch + 2], pk[8 * part + 4 * ch + 3]);
+      } else {
         const uint32_t rowaddr = smem_u32(sP) + row * 128;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch)
@@ -1147,15 +1243,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                        pk[4 * ch + 2], pk[4 * ch + 3]);
       }
       // rows past the sequence end: zero the V rows so 0 * (stale or NaN) never
-      // reaches the accumulator (warpgroup 0: head dims 0-127, 1: 128-255)
+      // reaches the accumulator (warpgroup 0: head dims 0-127, 1: 128-255;
+      // bf16: the item of those dims, two 64-dim regions; FP8: that half of
+      // the tensor's one item)
       if (valid < kTile) {
-        const uint32_t it = v_item(g, t.cta_last) + wg;
-        uint64_t* ready = kFp8 ? c.conv_full : c.slot_full;  // zero after the FP8 expansion
-        if (!warp_wait(&ready[it % kSlots], par(it / kSlots), abort_flag)) break;
+        const uint32_t it = v_item<kFp8>(g, t.cta_last) + (kFp8 ? 0 : wg);
+        if (!warp_wait(&c.slot_full[it % kSlots], par(it / kSlots), abort_flag)) break;
         if (!row_ok) {
-          const uint32_t base = smem_u32(sRing) + (it % kSlots) * kSlotBytes + row * 128;
+          const uint32_t base = smem_u32(sRing) + (it % kSlots) * kSlotBytes + row * 128 +
+                                (kFp8 ? wg * (kSlotBytes / 2) : 0);
 #pragma unroll
-          for (int r = 0; r < 2; ++r)
+          for (int r = 0; r < (kFp8 ? 1 : 2); ++r)
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
               st_shared_v4(base + r * (kSlotBytes / 2) + ch * 16, 0u, 0u, 0u, 0u);

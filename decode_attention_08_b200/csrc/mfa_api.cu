@@ -112,17 +112,22 @@ CUresult encode_3d(CUtensorMap* map, CUtensorMapDataType type, int esize, const 
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-// bf16 cache [B][L][256] (or page pool [P][page_size][256]) viewed as
-// {64 dims, tokens, 4 chunks, B or P} (strides: token, 128 B, sequence or page)
-// so one box of {64, 128, 2, 1} fills a 32 KB half-slot as two 128-row regions.
-CUresult encode_kv_chunked(CUtensorMap* map, const void* base, uint64_t tokens, uint64_t batch,
+// Cache [B][L][256] (or page pool [P][page_size][256]) with each 512-byte
+// (bf16) or 256-byte (E4M3) token row viewed as 128-byte chunks placed after
+// the token dimension: {chunk elements, tokens, chunks, B or P} (strides:
+// token, 128 B, sequence or page). One box of {chunk, 128, 2, 1} lands as two
+// 128-row regions of 16 KB: for bf16 one item (head dims 0-127 or 128-255),
+// for E4M3 the whole tensor tile.
+CUresult encode_kv_chunked(CUtensorMap* map, CUtensorMapDataType type, int esize,
+                           const void* base, uint64_t tokens, uint64_t batch,
                            uint64_t token_stride_elems, uint64_t batch_stride_elems) {
-  const cuuint64_t dims[4] = {64, tokens, 4, batch};
-  const cuuint64_t strides[3] = {token_stride_elems * 2, 128, batch_stride_elems * 2};
-  const cuuint32_t box[4] = {64, 128, 2, 1};
+  const cuuint64_t inner = 128 / esize;
+  const cuuint64_t dims[4] = {inner, tokens, kDim / inner, batch};
+  const cuuint64_t strides[3] = {token_stride_elems * esize, 128, batch_stride_elems * esize};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(inner), 128, 2, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return g_encode(map, type, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
@@ -410,13 +415,13 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
   const CUtensorMapDataType kv_type =
       fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint32_t box0 = fp8 ? 128 : 64;
-  if (!fp8 && rows == kTile) {
-    // bf16 contiguous, or pages of >= 128 tokens: tokens = cap or page_size,
-    // outer index = sequence or page
-    if (encode_kv_chunked(&tk, k_cache->data, d1s, d2, k_cache->stride[1], k_cache->stride[0]) !=
-            CUDA_SUCCESS ||
-        encode_kv_chunked(&tv, v_cache->data, d1s, d2, v_cache->stride[1], v_cache->stride[0]) !=
-            CUDA_SUCCESS)
+  if (rows == kTile) {
+    // contiguous, or pages of >= 128 tokens: tokens = cap or page_size, outer
+    // index = sequence or page
+    if (encode_kv_chunked(&tk, kv_type, esz, k_cache->data, d1s, d2, k_cache->stride[1],
+                          k_cache->stride[0]) != CUDA_SUCCESS ||
+        encode_kv_chunked(&tv, kv_type, esz, v_cache->data, d1s, d2, v_cache->stride[1],
+                          v_cache->stride[0]) != CUDA_SUCCESS)
       return MFA_ERR_INVALID_ARG;
   } else if (encode_3d(&tk, kv_type, esz, k_cache->data, kDim, d1s, d2, k_cache->stride[1],
                        k_cache->stride[0], box0, rows) != CUDA_SUCCESS ||

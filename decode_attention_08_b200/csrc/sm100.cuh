@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 namespace mfa {
 
@@ -219,6 +220,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The same descriptor with the 64-byte swizzle (8 rows of 64 bytes per atom).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
+  return d;
+}
+
 // Instruction descriptor of a dense kind::f16 MMA with fp32 accumulation.
 // ab_fmt: 0 = f16, 1 = bf16. a_mn/b_mn: 1 if that operand is MN-major.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_fmt, int a_mn, int b_mn) {
@@ -240,6 +252,34 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// As mma_f16_ss for 8-bit operands (kind::f8f6f4; with the descriptor's format
+// fields 0, both E4M3). The instruction descriptor has the kind::f16 layout.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Two values, each written exactly as the sum of two E4M3 numbers when it has
+// at most 8 significant bits and lies in E4M3's normal range (hi: the value
+// rounded to E4M3, lo: the remainder rounded to E4M3; the remainder of an
+// 8-bit significand keeps at most 4 bits). Returns hi in bits 0-15 and lo in
+// bits 16-31, the first value in the low byte of each.
+__device__ __forceinline__ uint32_t split_e4m3x2(float a, float b) {
+  const __half2 x = __floats2half2_rn(a, b);
+  const __nv_fp8x2_storage_t hi =
+      __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(x), __NV_SATFINITE, __NV_E4M3);
+  const __half2 hx = static_cast<__half2>(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3));
+  const __half2 r = __hsub2(x, hx);
+  const __nv_fp8x2_storage_t lo =
+      __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(r), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(hi) | (static_cast<uint32_t>(lo) << 16);
 }
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued before
