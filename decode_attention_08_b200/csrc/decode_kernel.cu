@@ -123,6 +123,17 @@ constexpr uint32_t kColObuf = 256; // column offset of the odd segments' O pair
 
 __device__ __forceinline__ uint32_t o_cols(int seg) { return (seg & 1) ? kColObuf : 0u; }
 
+// First column of O^T rows 128 r .. 128 r + 127 (r: head-dim half) for the
+// segment with ordinal seg. bf16: 64 columns (heads), double-buffered by
+// segment. FP8: 128 columns, the products with P's hi part in the first 64
+// and with its lo part in the next 64 (one N = 128 product per step reads each
+// V step once for both parts); single-buffered, so an FP8 segment's output is
+// read out at its end.
+template <bool kFp8>
+__device__ __forceinline__ uint32_t o_base(int seg, int r) {
+  return kFp8 ? (r ? 384u : 128u) : o_cols(seg) + (r ? kColOhi : kColOlo);
+}
+
 // Score buffer of tile g. bf16: 64 columns (heads). FP8: 128 columns, K.q_hi
 // in 0-63 and K.q_lo in 64-127 (one N = 128 product per step reads each K
 // step once for both parts).
@@ -859,7 +870,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // products of E4M3 operands straight from the ring (K, V), with q and P
     // each given as an exact E4M3 pair hi + lo (two products per step).
     constexpr uint32_t idesc_qk = idesc_f16(128, kFp8 ? 128 : 64, kFp8 ? 0 : 1, 0, 0);
-    constexpr uint32_t idesc_pv = idesc_f16(128, 64, kFp8 ? 0 : 1, 1, 1);
+    constexpr uint32_t idesc_pv = idesc_f16(128, kFp8 ? 128 : 64, kFp8 ? 0 : 1, 1, 1);
     constexpr uint32_t kIPT = kItemsPerTensor<kFp8>;
     const uint32_t q_base = smem_u32(sQ);
     const uint32_t ring_base = smem_u32(sRing);
@@ -885,38 +896,36 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       tc_fence_after();
       if (lane == 0) {
         MFA_TR(3, j);
-        const uint32_t d_o = tmem + o_cols(t.seg);
         if (kFp8) {
           // V slot: head dims 0-127 | 128-255, each 128 token rows of 128 B
-          // (MN-major A); P hi | lo: 128 token rows of 64 B (MN-major B)
+          // (MN-major A); P: 128 token rows of hi (64 B) and lo (64 B) as two
+          // 64-byte-swizzled blocks 8 KB apart (one N = 128 MN-major B)
           const uint32_t v = ring_base + (lo % kSlots) * kSlotBytes;
 #pragma unroll
-          for (int r = 0; r < 2; ++r)
+          for (int kk = 0; kk < kTile / 32; ++kk)
 #pragma unroll
-            for (int kk = 0; kk < kTile / 32; ++kk)
-#pragma unroll
-              for (int part = 0; part < 2; ++part)
-                mma_f8_ss(d_o + (r ? kColOhi : kColOlo),
-                          sw128_desc(v + r * (kSlotBytes / 2) + kk * 4096, kSlotBytes / 2, 1024),
-                          sw64_desc(p_base + part * (kPBytes / 2) + kk * 2048, kPBytes / 2, 512),
-                          idesc_pv, (t.seg_first && kk == 0 && part == 0) ? 0u : 1u);
+            for (int r = 0; r < 2; ++r)
+              mma_f8_ss(tmem + o_base<kFp8>(t.seg, r),
+                        sw128_desc(v + r * (kSlotBytes / 2) + kk * 4096, kSlotBytes / 2, 1024),
+                        sw64_desc(p_base + kk * 2048, kPBytes / 2, 512), idesc_pv,
+                        (t.seg_first && kk == 0) ? 0u : 1u);
           mma_commit(&c.slot_empty[lo % kSlots]);
         } else {
           const uint32_t hi = lo + 1;
           const uint32_t v_lo = ring_base + (lo % kSlots) * kSlotBytes;
           const uint32_t v_hi = ring_base + (hi % kSlots) * kSlotBytes;
-          // head dims 0-127 first, so their ring slot is released half-way
+          // the two head-dim halves accumulate into different columns: issue
+          // them alternately, so consecutive products do not wait on each other
 #pragma unroll
-          for (int s = 0; s < kTile / 16; ++s)
-            mma_f16_ss(d_o + kColOlo, sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
+          for (int s = 0; s < kTile / 16; ++s) {
+            mma_f16_ss(tmem + o_base<kFp8>(t.seg, 0), sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
                        sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
                        (t.seg_first && s == 0) ? 0u : 1u);
+            mma_f16_ss(tmem + o_base<kFp8>(t.seg, 1), sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
+                       sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                       (t.seg_first && s == 0) ? 0u : 1u);
+          }
           mma_commit(&c.slot_empty[lo % kSlots]);
-#pragma unroll
-          for (int s = 0; s < kTile / 16; ++s)
-            mma_f16_ss(d_o + kColOhi, sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
-                       sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
-                       (t.seg_first && s == 0) ? 0u : 1u);
           mma_commit(&c.slot_empty[hi % kSlots]);
         }
         mma_commit(&c.o_full);
@@ -1084,8 +1093,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       for (int half = 0; half < 2; ++half) {
         const int d = half * 128 + row;
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + o_cols(pt.seg) + (half ? kColOhi : kColOlo) + hbase, r);
-        tmem_wait_ld();
+        const uint32_t col = tmem + lane_addr + o_base<kFp8>(pt.seg, half) + hbase;
+        tmem_ld32(col, r);
+        if (kFp8) {  // O = (V P_hi) + (V P_lo)
+          uint32_t r2[32];
+          tmem_ld32(col + 64, r2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
+        } else {
+          tmem_wait_ld();
+        }
         if (pt.slot >= 0) {
           // partial layout [slot][head][d]: a warp writes 128 contiguous bytes per head
           float* dst = p.ws_o + static_cast<int64_t>(pt.slot) * kPartialFloats +
@@ -1210,11 +1229,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       tc_fence_after();
       if (rescale && !t.seg_first) {
 #pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {  // (O_lo, O_hi) x two 16-column chunks
+        for (int q4 = 0; q4 < (kFp8 ? 8 : 4); ++q4) {  // halves x two 16-column chunks (x 2 parts)
           uint32_t r[16];
           const int cb = (q4 & 1) * 16;
-          const uint32_t a =
-              tmem + lane_addr + o_cols(t.seg) + ((q4 >> 1) ? kColOhi : kColOlo) + hbase + cb;
+          const uint32_t a = tmem + lane_addr + o_base<kFp8>(t.seg, (q4 >> 1) & 1) + (q4 >> 2) * 64 +
+                             hbase + cb;
           tmem_ld16(a, r);
           tmem_wait_ld();
 #pragma unroll
@@ -1303,6 +1322,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         pend = t;
         pend_g = g;
         have_pending = true;
+        if (kFp8 && !t.cta_last) {
+          // single O buffer: read out now, before the next segment's first PV
+          if (!warp_wait(&c.o_full, par(g), abort_flag)) break;
+          tc_fence_after();
+          write_segment(pend);
+          have_pending = false;
+        }
       }
       ++g;
     }
