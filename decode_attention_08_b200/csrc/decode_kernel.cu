@@ -395,12 +395,6 @@ __device__ __forceinline__ void st_ready4(unsigned long long* dst, unsigned long
       : "memory");
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* src) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(src) : "memory");
-  return v;
-}
-
 // Publishes the end of a segment to the combine kernel (one thread). For a
 // split sequence the call counts as one of `arrivals` x (segments) arrivals;
 // the last one (after whose arrival every partial is in memory: each arriver
@@ -646,6 +640,131 @@ __device__ __forceinline__ float q_to_e4m3(uint32_t base, int lane) {
   return inv_s;
 }
 
+constexpr int kCombineHeads = 16;  // heads per CTA
+constexpr int kCombineDims = 16;   // head-dim elements per thread (kDim / 16 threads per head)
+constexpr int kCombineBatch = 4;   // partials loaded per round trip
+
+// Waits (bounded) until *w is non-zero; returns it, or 0 after the wait limit.
+// Polls with plain volatile loads; the fence after the last one makes it an
+// acquire, ordering the caller's reads of the partials after the word.
+__device__ unsigned long long wait_ready(const unsigned long long* w) {
+  const volatile unsigned long long* vw = w;
+  unsigned long long v = *vw;
+  if (v == 0) {
+    const uint64_t t0 = global_timer_ns();
+    while ((v = *vw) == 0) {
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        record_error(6 /* MFA_ERR_TIMEOUT */);
+        return 0;
+      }
+    }
+  }
+  __threadfence();
+  return v;
+}
+
+// 16 consecutive output elements of (b, h) from d0 (16-byte vector stores
+// when the address allows).
+__device__ __forceinline__ void store_out16(const DecodeParams& p, int b, int h, int d0,
+                                            const float* v) {
+  const int64_t off = static_cast<int64_t>(b) * p.out_sb + static_cast<int64_t>(h) * p.out_sh + d0;
+  if (p.out_f32) {
+    float* dst = static_cast<float*>(p.out) + off;
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+      for (int j = 0; j < kCombineDims / 4; ++j)
+        reinterpret_cast<float4*>(dst)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kCombineDims; ++j) dst[j] = v[j];
+    }
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + off;
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+      for (int j = 0; j < kCombineDims / 8; ++j)
+        reinterpret_cast<uint4*>(dst)[j] =
+            make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                       pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < kCombineDims; ++j) dst[j] = __float2bfloat16_rn(v[j]);
+    }
+  }
+}
+
+// Merges the partials of split sequence b for head h, head-dim elements
+// d0 .. d0 + 15, in plan order (up to four per round trip), and writes the
+// output and (d0 == 0) the log-sum-exp. The partials must be visible to the
+// caller (acquired after the sequence's last arrival).
+__device__ __forceinline__ void merge_head_part(const DecodeParams& p, int b, const SplitList& sl,
+                                                int h, int d0) {
+  // online merge: running max m, running weight sum l, running weighted sums v
+  float v[kCombineDims];
+  float m = -INFINITY, l = 0.f;
+#pragma unroll
+  for (int j = 0; j < kCombineDims; ++j) v[j] = 0.f;
+  for (int i = 0; i < sl.count; i += kCombineBatch) {
+    int slot[kCombineBatch];
+    bool any = false;
+#pragma unroll
+    for (int k = 0; k < kCombineBatch; ++k) {
+      slot[k] = i + k < sl.count ? sl.slot(i + k) : -1;
+      any |= slot[k] >= 0;
+    }
+    if (!any) continue;  // empty units of a fixed split
+    float e[kCombineBatch];
+    float4 o[kCombineBatch][kCombineDims / 4];
+#pragma unroll
+    for (int k = 0; k < kCombineBatch; ++k) {
+      const int sk = slot[k] < 0 ? 0 : slot[k];
+      const float4* src = reinterpret_cast<const float4*>(
+          p.ws_o + static_cast<int64_t>(sk) * kPartialFloats + static_cast<int64_t>(h) * kDim + d0);
+      e[k] = slot[k] >= 0 ? __ldcg(p.ws_lse + static_cast<int64_t>(sk) * kHeads + h) : -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kCombineDims / 4; ++j)
+        o[k][j] = slot[k] >= 0 ? __ldcg(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float mn = m;
+#pragma unroll
+    for (int k = 0; k < kCombineBatch; ++k) mn = fmaxf(mn, e[k]);  // finite: one slot is valid
+    const float c = ex2_approx((m - mn) * kLog2e);
+    l *= c;
+#pragma unroll
+    for (int j = 0; j < kCombineDims; ++j) v[j] *= c;
+#pragma unroll
+    for (int k = 0; k < kCombineBatch; ++k) {
+      const float w = ex2_approx((e[k] - mn) * kLog2e);
+      l += w;
+#pragma unroll
+      for (int j = 0; j < kCombineDims / 4; ++j) {
+        v[4 * j] += w * o[k][j].x;
+        v[4 * j + 1] += w * o[k][j].y;
+        v[4 * j + 2] += w * o[k][j].z;
+        v[4 * j + 3] += w * o[k][j].w;
+      }
+    }
+    m = mn;
+  }
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int j = 0; j < kCombineDims; ++j) v[j] *= inv;
+  store_out16(p, b, h, d0, v);
+  if (p.lse_out && d0 == 0) p.lse_out[b * p.lse_sb + h] = m + lg2_approx(l) * kLn2;
+}
+
+// The split list of sequence b from its ready word (state kReadyMerge).
+__device__ __forceinline__ SplitList split_list_of(const DecodeParams& p, int b, int nt,
+                                                   unsigned long long word) {
+  SplitList sl;
+  if (p.num_splits == 0)
+    sl.init_balanced(static_cast<long long>((word & 0xffffffffull) >> 2), nt,
+                     static_cast<long long>(word >> 32), p.grid);
+  else
+    sl.init_fixed(b, nt, p.num_splits);
+  return sl;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -711,6 +830,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     tma_prefetch_desc(&tm_v);
   }
 
+  // ---- warm L2 while the previous kernel finishes ---------------------------
+  // This call's inputs may not be read before the dependency wait, but an L2
+  // prefetch changes no result: the first K/V tiles this CTA took in the
+  // previous call on this workspace (a decode loop's plan barely moves from
+  // step to step) are fetched while HBM idles under the previous kernel's tail.
+  if (!kPaged && p.num_splits == 0 && warp == 0 && lane == 0) {
+    const int hb = *reinterpret_cast<volatile const int*>(p.ws_hint + 2 * blockIdx.x);
+    const int ht = *reinterpret_cast<volatile const int*>(p.ws_hint + 2 * blockIdx.x + 1);
+    if (hb >= 0 && hb < p.batch && ht >= 0 && ht < (p.cap_tokens + kTile - 1) / kTile) {
+      for (int i = 0; i < 2; ++i)
+        for (int ch = 0; ch < (kFp8 ? 1 : 2); ++ch) {
+          tma_prefetch_4d(&tm_k, 0, (ht + i) * kTile, 2 * ch, hb);
+          tma_prefetch_4d(&tm_v, 0, (ht + i) * kTile, 2 * ch, hb);
+        }
+    }
+  }
+
   // ---- plan (reads seq_lens: after the previous kernel has completed) -----
   griddep_wait();
   // The combine kernel may start from here on: it waits for each sequence's
@@ -730,6 +866,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   __syncthreads();
   if (p.num_splits == 0) {
     balanced_plan(p, c, lens_s);  // ends with __syncthreads
+    if (tid == 0) {  // the next call's L2 warm-up hint
+      p.ws_hint[2 * blockIdx.x] = c.tiles > 0 ? c.b_start : -1;
+      p.ws_hint[2 * blockIdx.x + 1] = c.off_start;
+    }
   } else if (tid == 0) {
     c.tiles = static_cast<int>(blockIdx.x) < p.batch * p.num_splits ? -1 : 0;
     c.t0 = 0;
@@ -1366,55 +1506,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 // for the attention grid to complete only at its end, so a call is over when
 // this kernel is.
 // ===========================================================================
-constexpr int kCombineHeads = 16;  // heads per CTA
-constexpr int kCombineDims = 16;   // head-dim elements per thread (kDim / 16 threads per head)
-constexpr int kCombineBatch = 4;   // partials loaded per round trip
-
-// Waits (bounded) until *w is non-zero; returns it, or 0 after the wait limit.
-__device__ unsigned long long wait_ready(const unsigned long long* w) {
-  unsigned long long v = ld_acquire_u64(w);
-  if (v != 0) return v;
-  const uint64_t t0 = global_timer_ns();
-  while ((v = ld_acquire_u64(w)) == 0) {
-    __nanosleep(128);
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      record_error(6 /* MFA_ERR_TIMEOUT */);
-      return 0;
-    }
-  }
-  return v;
-}
-
-// 16 consecutive output elements of (b, h) from d0 (16-byte vector stores
-// when the address allows).
-__device__ __forceinline__ void store_out16(const DecodeParams& p, int b, int h, int d0,
-                                            const float* v) {
-  const int64_t off = static_cast<int64_t>(b) * p.out_sb + static_cast<int64_t>(h) * p.out_sh + d0;
-  if (p.out_f32) {
-    float* dst = static_cast<float*>(p.out) + off;
-    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-#pragma unroll
-      for (int j = 0; j < kCombineDims / 4; ++j)
-        reinterpret_cast<float4*>(dst)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < kCombineDims; ++j) dst[j] = v[j];
-    }
-  } else {
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + off;
-    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-#pragma unroll
-      for (int j = 0; j < kCombineDims / 8; ++j)
-        reinterpret_cast<uint4*>(dst)[j] =
-            make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                       pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-    } else {
-#pragma unroll
-      for (int j = 0; j < kCombineDims; ++j) dst[j] = __float2bfloat16_rn(v[j]);
-    }
-  }
-}
-
 __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams p) {
 #ifdef MFA_TRACE
   const unsigned long long gt_start = global_timer_ns();
@@ -1460,65 +1551,7 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
     store_out16(p, b, h, d0, v);
     if (p.lse_out && d0 == 0) p.lse_out[b * p.lse_sb + h] = -INFINITY;
   } else if ((word & 3) == kReadyMerge) {
-    SplitList sl;
-    if (p.num_splits == 0)
-      sl.init_balanced(static_cast<long long>((word & 0xffffffffull) >> 2), nt,
-                       static_cast<long long>(word >> 32), p.grid);
-    else
-      sl.init_fixed(b, nt, p.num_splits);
-
-    // online merge in plan order, up to four partials per step: running max
-    // m, running weight sum l and running weighted sums acc of this head
-    float m = -INFINITY, l = 0.f;
-#pragma unroll
-    for (int j = 0; j < kCombineDims; ++j) v[j] = 0.f;
-    for (int i = 0; i < sl.count; i += kCombineBatch) {
-      int slot[kCombineBatch];
-      bool any = false;
-#pragma unroll
-      for (int k = 0; k < kCombineBatch; ++k) {
-        slot[k] = i + k < sl.count ? sl.slot(i + k) : -1;
-        any |= slot[k] >= 0;
-      }
-      if (!any) continue;  // empty units of a fixed split
-      float e[kCombineBatch];
-      float4 o[kCombineBatch][kCombineDims / 4];
-#pragma unroll
-      for (int k = 0; k < kCombineBatch; ++k) {
-        const int sk = slot[k] < 0 ? 0 : slot[k];
-        const float4* src = reinterpret_cast<const float4*>(
-            p.ws_o + static_cast<int64_t>(sk) * kPartialFloats + static_cast<int64_t>(h) * kDim + d0);
-        e[k] = slot[k] >= 0 ? __ldcg(p.ws_lse + static_cast<int64_t>(sk) * kHeads + h) : -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kCombineDims / 4; ++j)
-          o[k][j] = slot[k] >= 0 ? __ldcg(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      float mn = m;
-#pragma unroll
-      for (int k = 0; k < kCombineBatch; ++k) mn = fmaxf(mn, e[k]);  // finite: one slot is valid
-      const float c = ex2_approx((m - mn) * kLog2e);
-      l *= c;
-#pragma unroll
-      for (int j = 0; j < kCombineDims; ++j) v[j] *= c;
-#pragma unroll
-      for (int k = 0; k < kCombineBatch; ++k) {
-        const float w = ex2_approx((e[k] - mn) * kLog2e);
-        l += w;
-#pragma unroll
-        for (int j = 0; j < kCombineDims / 4; ++j) {
-          v[4 * j] += w * o[k][j].x;
-          v[4 * j + 1] += w * o[k][j].y;
-          v[4 * j + 2] += w * o[k][j].z;
-          v[4 * j + 3] += w * o[k][j].w;
-        }
-      }
-      m = mn;
-    }
-    const float inv = 1.f / l;
-#pragma unroll
-    for (int j = 0; j < kCombineDims; ++j) v[j] *= inv;
-    store_out16(p, b, h, d0, v);
-    if (p.lse_out && d0 == 0) p.lse_out[b * p.lse_sb + h] = m + lg2_approx(l) * kLn2;
+    merge_head_part(p, b, split_list_of(p, b, nt, word), h, d0);
   }
   // back to zero for the next call, which sets it only after this kernel
   // has completed

@@ -213,7 +213,7 @@ bool sync_words_stale(const void* ws, int batch) {
 // attention and the combine kernel (an arrival counter, four ready words),
 // then the partial outputs of split sequences and their log-sum-exp values.
 struct DecodeWsLayout {
-  size_t arrive_off, ready_off, sync_bytes, o_off, lse_off, total;
+  size_t arrive_off, ready_off, sync_bytes, o_off, lse_off, hint_off, total;
   int slots;
 };
 
@@ -226,7 +226,8 @@ DecodeWsLayout decode_ws_layout(int batch, int num_splits, int grid) {
   l.sync_bytes = align256(l.ready_off + B * 4 * sizeof(unsigned long long));
   l.o_off = l.sync_bytes;
   l.lse_off = align256(l.o_off + static_cast<size_t>(l.slots) * kPartialFloats * sizeof(float));
-  l.total = align256(l.lse_off + static_cast<size_t>(l.slots) * kHeads * sizeof(float));
+  l.hint_off = align256(l.lse_off + static_cast<size_t>(l.slots) * kHeads * sizeof(float));
+  l.total = align256(l.hint_off + static_cast<size_t>(grid) * 2 * sizeof(int));
   return l;
 }
 
@@ -454,6 +455,7 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
   p.ws_lse = reinterpret_cast<float*>(ws + wl.lse_off);
+  p.ws_hint = reinterpret_cast<int*>(ws + wl.hint_off);
   p.ws_arrive = reinterpret_cast<unsigned*>(ws + wl.arrive_off);
   p.ws_ready = reinterpret_cast<unsigned long long*>(ws + wl.ready_off);
 

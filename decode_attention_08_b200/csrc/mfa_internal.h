@@ -55,6 +55,10 @@ struct DecodeParams {
   // pending, kReadyNone, kReadyMerge), bits 2-31 the sequence's first global
   // tile, bits 32-63 the batch's total tiles (balanced plan)
   unsigned long long* ws_ready;
+  // [grid][2] where each CTA's tiles began in the previous call on this
+  // workspace (first sequence, first tile): a hint for warming L2 before the
+  // call's inputs may be read; never trusted for results
+  int* ws_hint;
 };
 
 constexpr unsigned kReadyNone = 1;   // the attention kernel wrote the sequence's output itself
