@@ -230,7 +230,7 @@ class DecodeStep:
                                      k_scale=self.dec.k_scale, v_scale=self.dec.v_scale,
                                      num_splits=self.num_splits, workspace=self.ws)
 
-    def capture(self, steps_per_graph: int = 6):
+    def capture(self, steps_per_graph: int = 10):
         """One graph per rotating cache copy holding a single step, plus graphs
         of `steps_per_graph` consecutive steps (copies rotating inside) so that
         consecutive steps overlap through programmatic dependent launch."""
@@ -448,7 +448,7 @@ def time_qproj(proj: gen.ProjInputs, hbm_peak: float):
     flops = 2 * x.shape[0] * (wa.numel() + wb.numel())
     return {"us_per_call": t * 1e6, "alg_bytes": alg, "gbs": alg / t / 1e9,
             "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak, "tflops": flops / t / 1e12,
-            "note": "two launches (latent GEMM with split-K merge, up-projection GEMM)"}
+            "note": "batch <= 8: one persistent kernel (split-K latent GEMM, deterministic merge, up-projection whose weights fill the ring while the latent forms); larger batches: two launches"}
 
 
 def run_ours(args, world, rank, local):

@@ -15,6 +15,10 @@ int decode_smem_bytes();
 cudaError_t launch_decode(bool paged, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                           const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);
 int qproj_smem_bytes(int n_cols);
+bool qproj_fused_fits(int n1, int n2, int k2_blocks);
+cudaError_t launch_qproj_fused(const CUtensorMap& twa, const CUtensorMap& tx,
+                               const CUtensorMap& twb, const CUtensorMap& tl,
+                               const QprojFusedParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_qproj(const CUtensorMap& tw, const CUtensorMap& ta, const QprojParams& p,
                          int m_tiles, cudaStream_t stream);
 }  // namespace mfa
@@ -138,6 +142,20 @@ CUresult encode_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
   const cuuint32_t box[2] = {b0, b1};
   const cuuint32_t estr[2] = {1, 1};
   return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// Row-major weight [K][N] viewed as {64 features, K, N / 64 feature chunks}
+// (strides: row, 128 B): one box of {64, 64, 2} is a 128-feature x 64-k tile,
+// landing as its two 64-feature halves 8 KB apart (one TMA op per stage).
+CUresult encode_w3d(CUtensorMap* map, const void* base, uint64_t n, uint64_t k,
+                    uint64_t row_stride_elems) {
+  const cuuint64_t dims[3] = {64, k, n / 64};
+  const cuuint64_t strides[2] = {row_stride_elems * 2, 128};
+  const cuuint32_t box[3] = {64, 64, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
@@ -551,6 +569,36 @@ int qproj_impl(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_
       encode_2d(&tl, latent, R, 2 * B, R, 64, n2) != CUDA_SUCCESS)
     return MFA_ERR_INVALID_ARG;
 
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int m1 = static_cast<int>(R / 128), m2 = static_cast<int>(N / 128);
+  if (B <= 8 && m1 < kQprojDone && m1 * wl.splits <= dev.sms && m2 <= dev.sms &&
+      qproj_fused_fits(n1, n2, static_cast<int>(R / 64))) {
+    // both GEMMs in one persistent kernel (see qproj_kernel.cu)
+    QprojFusedParams pf;
+    std::memset(&pf, 0, sizeof pf);
+    pf.batch = static_cast<int>(B);
+    pf.k1_blocks = static_cast<int>(Dm / 64);
+    pf.k2_blocks = static_cast<int>(R / 64);
+    pf.m1_tiles = m1;
+    pf.m2_tiles = m2;
+    pf.splits = wl.splits;
+    pf.n1 = n1;
+    pf.n2 = n2;
+    pf.rank = static_cast<int>(R);
+    pf.partials = reinterpret_cast<float*>(ws + wl.part_off);
+    pf.counters = reinterpret_cast<int*>(ws + wl.cnt_off);
+    pf.latent = latent;
+    pf.q_out = static_cast<__nv_bfloat16*>(q_out->data);
+    pf.q_stride = q_out->stride[0];
+    CUtensorMap tw1v, tw2v;
+    if (encode_w3d(&tw1v, w_qa->data, R, Dm, w_qa->stride[0]) != CUDA_SUCCESS ||
+        encode_w3d(&tw2v, w_qb->data, N, R, w_qb->stride[0]) != CUDA_SUCCESS)
+      return MFA_ERR_INVALID_ARG;
+    const int grid = m1 * wl.splits > m2 ? m1 * wl.splits : m2;
+    const cudaError_t ef = launch_qproj_fused(tw1v, tx, tw2v, tl, pf, grid, st);
+    return ef == cudaSuccess ? MFA_OK : cuda_fail(ef);
+  }
+
   QprojParams p1;
   std::memset(&p1, 0, sizeof p1);
   p1.batch = static_cast<int>(B);
@@ -562,7 +610,6 @@ int qproj_impl(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_
   p1.partials = reinterpret_cast<float*>(ws + wl.part_off);
   p1.counters = reinterpret_cast<int*>(ws + wl.cnt_off);
   p1.latent = latent;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_qproj(tw1, tx, p1, static_cast<int>(R / 128), st);
   if (e != cudaSuccess) return cuda_fail(e);
 

@@ -78,4 +78,23 @@ struct QprojParams {
   int64_t q_stride;      // elements between q_out rows
 };
 
+// Both projection GEMMs in one persistent kernel (small batches): split-K
+// latent GEMM on m1_tiles x splits CTAs, then the up-projection on m2_tiles
+// CTAs, whose weights stream into L2 while the latent is still being formed.
+struct QprojFusedParams {
+  int batch;
+  int k1_blocks, k2_blocks;  // contraction lengths / 64 (hidden, rank)
+  int m1_tiles, m2_tiles;    // output tiles of 128 (rank, heads x dim)
+  int splits;                // split-K factor of the latent GEMM
+  int n1, n2;                // MMA N of the two GEMMs (batch, 2 x batch, padded to 16)
+  int rank;                  // latent width
+  float* partials;           // [splits][batch][rank]
+  int* counters;             // [m1_tiles] split arrivals; counters[kQprojDone]: latent tiles done
+  __nv_bfloat16* latent;     // [2 * batch][rank], rows 2j / 2j + 1 = high part / residual
+  __nv_bfloat16* q_out;
+  int64_t q_stride;
+};
+
+constexpr int kQprojDone = 1023;  // counter index of the fused kernel's latent-ready count
+
 }  // namespace mfa

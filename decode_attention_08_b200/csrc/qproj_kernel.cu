@@ -48,6 +48,42 @@ __host__ __device__ inline int gemm_tmem_cols(int n_cols) {
   return c;
 }
 
+
+// Deterministic split-K merge of latent feature m: for every row j, the sum
+// over splits in split order of partials[split][j][m], stored as a bf16 high
+// part (row 2j) and a bf16 residual (row 2j + 1). Loads for up to 16 splits
+// and kMergeRows rows are all issued before the first add, so the merge costs
+// a few L2 round trips rather than one per partial.
+constexpr int kMergeSplits = 16;
+
+template <int kMergeRows>
+__device__ __forceinline__ void merge_latent(const float* partials, int splits, int B,
+                                             int rank, int m, __nv_bfloat16* latent) {
+  for (int j0 = 0; j0 < B; j0 += kMergeRows) {
+    for (int s0 = 0; s0 < splits; s0 += kMergeSplits) {
+      float v[kMergeRows][kMergeSplits];
+#pragma unroll
+      for (int u = 0; u < kMergeSplits; ++u)
+#pragma unroll
+        for (int r = 0; r < kMergeRows; ++r)
+          v[r][u] = (s0 + u < splits && j0 + r < B)
+                        ? __ldcg(partials + (static_cast<int64_t>(s0 + u) * B + j0 + r) * rank + m)
+                        : 0.f;
+#pragma unroll
+      for (int r = 0; r < kMergeRows; ++r) {
+        if (j0 + r >= B) break;
+        float acc = s0 == 0 ? 0.f : __bfloat162float(latent[static_cast<int64_t>(2 * (j0 + r)) * rank + m]) +
+                                        __bfloat162float(latent[static_cast<int64_t>(2 * (j0 + r) + 1) * rank + m]);
+#pragma unroll
+        for (int u = 0; u < kMergeSplits; ++u) acc += v[r][u];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
+        latent[static_cast<int64_t>(2 * (j0 + r)) * rank + m] = hi;
+        latent[static_cast<int64_t>(2 * (j0 + r) + 1) * rank + m] = lo;
+      }
+    }
+  }
+}
 }  // namespace
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -173,18 +209,288 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     if (c.is_last) {
       __threadfence();
-      for (int j = 0; j < B; ++j) {
-        float acc = 0.f;
-        for (int s = 0; s < p.splits; ++s)
-          acc += __ldcg(p.partials + (static_cast<int64_t>(s) * B + j) * p.m_total + m);
-        const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
-        p.latent[static_cast<int64_t>(2 * j) * p.m_total + m] = hi;
-        p.latent[static_cast<int64_t>(2 * j + 1) * p.m_total + m] = lo;
-      }
+      merge_latent<2>(p.partials, p.splits, B, p.m_total, m, p.latent);
       if (tid == 0) p.counters[m_tile] = 0;
     }
   }
+}
+
+// ===========================================================================
+// Both GEMMs in one persistent kernel, for small batches. CTA i < m1_tiles x
+// splits computes a split-K part of the latent GEMM as above; CTA i <
+// m2_tiles owns output tile i of the up-projection. An up-projection stage
+// holds a weight tile and the matching 64-wide slice of the latent, loaded
+// separately: the weight parts are issued as soon as slots free, so the ring
+// fills with the second GEMM's weights while the latent is still being
+// formed, and the latent parts follow once every latent tile is complete (a
+// bounded wait on the latent-ready count, taken only when the ring is full).
+// Grid = at most one CTA per SM, so every CTA is resident while others wait.
+// The weights come through 3-D maps (64 features, k, 64-feature chunk): one
+// TMA op per 128 x 64 tile. Warp 0 loads, warp 1 issues the products; warps
+// 2-5 (TMEM lane quarters warp & 3) run the epilogues and synchronise only
+// among themselves.
+// ===========================================================================
+namespace {
+
+constexpr int kFusedThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kFusedTmemCols = 64;  // latent accumulator at 0, output accumulator at 32
+
+__device__ __forceinline__ void epi_sync() {  // warps 2-5 only
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
+struct __align__(8) FusedCtrl {
+  uint64_t full[16], empty[16];
+  uint64_t acc1, acc2;
+  uint32_t tmem_base;
+  int abort_flag;
+  int is_last;
+};
+
+__host__ __device__ inline int fused_stage_bytes(int n1, int n2) {
+  return kABytes + (n1 > n2 ? n1 : n2) * 128;
+}
+
+__host__ __device__ inline int fused_stages(int stage_bytes) {
+  const int s = (218 * 1024) / stage_bytes;
+  return s > 16 ? 16 : s;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    mfa_qproj_fused_kernel(const __grid_constant__ CUtensorMap tm_wa,
+                           const __grid_constant__ CUtensorMap tm_x,
+                           const __grid_constant__ CUtensorMap tm_wb,
+                           const __grid_constant__ CUtensorMap tm_lat, const QprojFusedParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int stage_bytes = fused_stage_bytes(p.n1, p.n2);
+  const int stages = fused_stages(stage_bytes);
+  FusedCtrl& c = *reinterpret_cast<FusedCtrl*>(smem + stages * stage_bytes);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool has1 = static_cast<int>(blockIdx.x) < p.m1_tiles * p.splits;
+  const int tile1 = blockIdx.x % p.m1_tiles;
+  const int split = blockIdx.x / p.m1_tiles;
+  const int kb0 = static_cast<int>((static_cast<long long>(split) * p.k1_blocks) / p.splits);
+  const int kb1 = static_cast<int>((static_cast<long long>(split + 1) * p.k1_blocks) / p.splits);
+  const bool has2 = static_cast<int>(blockIdx.x) < p.m2_tiles;
+  const int tile2 = blockIdx.x;
+
+  if (tid == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&c.full[i], 1);
+      mbar_init(&c.empty[i], 1);
+    }
+    mbar_init(&c.acc1, 1);
+    mbar_init(&c.acc2, 1);
+    c.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&c.tmem_base, kFusedTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  volatile int* abort_flag = &c.abort_flag;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer ----------------
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_a = l2_policy_evict_last();
+    tma_prefetch_desc(&tm_wa);
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_wb);
+    tma_prefetch_desc(&tm_lat);
+    int i = 0;
+    bool ok = true;
+    if (has1) {
+      for (int kb = kb0; kb < kb1; ++kb, ++i) {
+        const int s = i % stages;
+        if (!(ok = mbar_wait(&c.empty[s], ((i / stages) & 1) ^ 1, abort_flag))) break;
+        uint8_t* st = smem + s * stage_bytes;
+        mbar_arrive_expect_tx(&c.full[s], kABytes + p.n1 * 128);
+        tma_load_3d(st, &tm_wa, &c.full[s], 0, kb * 64, 2 * tile1, pol_w);
+        tma_load_2d(st + kABytes, &tm_x, &c.full[s], kb * 64, 0, pol_a);
+      }
+    }
+    if (has2 && ok) {
+      const int i2 = i;   // stage counter of the first up-projection k-block
+      int lat_issued = 0;  // k-blocks whose latent part is issued
+      bool lat_ready = false;
+      // latent parts of k-blocks [lat_issued, kb_end)
+      auto issue_latent = [&](int kb_end) {
+        for (; lat_issued < kb_end; ++lat_issued) {
+          const int s = (i2 + lat_issued) % stages;
+          tma_load_2d(smem + s * stage_bytes + kABytes, &tm_lat, &c.full[s], lat_issued * 64, 0,
+                      pol_a);
+        }
+      };
+      // the whole latent exists once every latent tile is merged (bounded)
+      auto await_latent = [&]() -> bool {
+        volatile int* done = p.counters + kQprojDone;
+        const uint64_t t0 = global_timer_ns();
+        while (*done < p.m1_tiles) {
+          if (*abort_flag) return false;
+          if (global_timer_ns() - t0 > kWaitLimitNs) {
+            record_error(6 /* MFA_ERR_TIMEOUT */);
+            *abort_flag = 1;
+            return false;
+          }
+        }
+        __threadfence();             // acquire the latent tiles
+        fence_proxy_async_global();  // ... for the TMA reads that follow
+        // count this CTA as having seen the latent; the last one (after all
+        // latent tiles and every other reader) returns the count to zero
+        if (atomicAdd(p.counters + kQprojDone, 1) == p.m1_tiles + p.m2_tiles - 1)
+          p.counters[kQprojDone] = 0;
+        return true;
+      };
+      for (int kb = 0; kb < p.k2_blocks && ok; ++kb, ++i) {
+        const int s = i % stages;
+        if (!lat_ready && kb >= stages) {
+          // the ring is full of weight parts: the products need the latent now
+          if (!(ok = await_latent())) break;
+          lat_ready = true;
+          issue_latent(kb);
+        }
+        if (!(ok = mbar_wait(&c.empty[s], ((i / stages) & 1) ^ 1, abort_flag))) break;
+        uint8_t* st = smem + s * stage_bytes;
+        mbar_arrive_expect_tx(&c.full[s], kABytes + p.n2 * 128);
+        tma_load_3d(st, &tm_wb, &c.full[s], 0, kb * 64, 2 * tile2, pol_w);
+        if (lat_ready) issue_latent(kb + 1);
+      }
+      if (ok && !lat_ready && await_latent()) issue_latent(p.k2_blocks);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t idesc1 = idesc_f16(128, p.n1, 1, 1, 0);
+    const uint32_t idesc2 = idesc_f16(128, p.n2, 1, 1, 0);
+    int i = 0;
+    bool ok = true;
+    if (has1) {
+      for (int kb = kb0; kb < kb1; ++kb, ++i) {
+        const int s = i % stages;
+        if (!(ok = mbar_wait(&c.full[s], (i / stages) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + s * stage_bytes);
+        const uint32_t b = a + kABytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_f16_ss(tmem, sw128_desc(a + k * 2048, kABytes / 2, 1024),
+                     sw128_desc(b + k * 32, 16, 1024), idesc1, (kb > kb0 || k > 0) ? 1u : 0u);
+        mma_commit(&c.empty[s]);
+      }
+      mma_commit(&c.acc1);
+    }
+    if (has2 && ok) {
+      for (int kb = 0; kb < p.k2_blocks; ++kb, ++i) {
+        const int s = i % stages;
+        if (!mbar_wait(&c.full[s], (i / stages) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + s * stage_bytes);
+        const uint32_t b = a + kABytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_f16_ss(tmem + 32, sw128_desc(a + k * 2048, kABytes / 2, 1024),
+                     sw128_desc(b + k * 32, 16, 1024), idesc2, (kb > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&c.empty[s]);
+      }
+    }
+    if (has2) mma_commit(&c.acc2);
+  }
+  __syncwarp();
+
+  // ---------------- epilogues: thread = output feature row ----------------
+  const int quarter = warp & 3;  // TMEM lanes 32 quarter .. 32 quarter + 31
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+  const int etid = tid - 64;     // 0 .. 127 in warps 2-5
+  const int B = p.batch;
+  if (warp >= 2 && has1) {
+    const bool ready = mbar_wait(&c.acc1, 0, abort_flag);
+    tc_fence_after();
+    const int m = tile1 * 128 + quarter * 32 + lane;
+    if (ready) {
+      for (int cb = 0; cb < p.n1; cb += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + cb, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (cb + j < B)
+            p.partials[(static_cast<int64_t>(split) * B + cb + j) * p.rank + m] =
+                __uint_as_float(r[j]);
+      }
+    }
+    // deterministic split-K merge by the last CTA of this latent tile
+    __threadfence();
+    epi_sync();
+    if (etid == 0) {
+      const int prev = atomicAdd(p.counters + tile1, 1);
+      c.is_last = (prev == p.splits - 1);
+    }
+    epi_sync();
+    if (c.is_last) {
+      __threadfence();
+      merge_latent<4>(p.partials, p.splits, B, p.rank, m, p.latent);
+      __threadfence();
+      epi_sync();
+      if (etid == 0) {
+        p.counters[tile1] = 0;
+        atomicAdd(p.counters + kQprojDone, 1);  // this latent tile is complete
+      }
+    }
+  }
+  if (warp >= 2 && has2) {
+    const bool ready = mbar_wait(&c.acc2, 0, abort_flag);
+    tc_fence_after();
+    const int m = tile2 * 128 + quarter * 32 + lane;
+    if (ready && !*abort_flag) {
+      // latent rows are interleaved (2j = high part, 2j+1 = residual)
+      for (int cb = 0; cb < p.n2; cb += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + 32 + cb, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int row = cb / 2 + jj;
+          if (row < B)
+            p.q_out[static_cast<int64_t>(row) * p.q_stride + m] =
+                __float2bfloat16_rn(__uint_as_float(r[2 * jj]) + __uint_as_float(r[2 * jj + 1]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, kFusedTmemCols);
+}
+
+int qproj_fused_smem_bytes(int n1, int n2) {
+  const int stage_bytes = fused_stage_bytes(n1, n2);
+  return fused_stages(stage_bytes) * stage_bytes + static_cast<int>(sizeof(FusedCtrl)) + 1024;
+}
+
+bool qproj_fused_fits(int n1, int n2, int k2_blocks) {
+  (void)k2_blocks;
+  return n1 <= 32 && n2 <= 32 && fused_stages(fused_stage_bytes(n1, n2)) >= 4;
+}
+
+cudaError_t launch_qproj_fused(const CUtensorMap& twa, const CUtensorMap& tx,
+                               const CUtensorMap& twb, const CUtensorMap& tl,
+                               const QprojFusedParams& p, int grid, cudaStream_t stream) {
+  const int smem = qproj_fused_smem_bytes(p.n1, p.n2);
+  cudaError_t err = cudaFuncSetAttribute(mfa_qproj_fused_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  mfa_qproj_fused_kernel<<<grid, kFusedThreads, smem, stream>>>(twa, tx, twb, tl, p);
+  return cudaGetLastError();
 }
 
 int qproj_smem_bytes(int n_cols) {

@@ -182,7 +182,10 @@ int mfa_query_proj(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor
 
 /* As mfa_query_proj with a caller workspace of at least
  * mfa_query_proj_workspace_size(B, Dm, R) bytes, 256-byte aligned, that must be
- * zero-filled before its first use; every call leaves it zero-filled again. */
+ * zero-filled before its first use; every call returns its counters (the first
+ * 4 KB) to zero, and the rest needs no initialisation. With B <= 8 both
+ * products run in one persistent kernel that streams W_qb into L2 while the
+ * latent is formed. */
 int mfa_query_proj_ex(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
                       mfa_tensor* q_out, void* workspace, size_t workspace_bytes,
                       mfa_stream_t stream);
