@@ -80,11 +80,11 @@ constexpr int kWGHeads = kHeads / kWG;
 // shared-memory control block
 // ---------------------------------------------------------------------------
 struct __align__(16) DecodeCtrl {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];  // per q buffer (FP8: two, alternating by segment)
   uint64_t slot_full[kSlots], slot_empty[kSlots];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, o_full;
-  uint64_t q_conv;  // FP8 cache: q converted to its E4M3 pair
+  uint64_t q_conv[2];  // FP8 cache: q buffer converted to its E4M3 pair
   uint64_t red_full[kWG][2], l_full[kWG];
   uint64_t drain;
   long long t0;    // first global tile of this CTA (balanced plan)
@@ -108,12 +108,24 @@ static_assert(offsetof(DecodeCtrl, red) % 16 == 0 && offsetof(DecodeCtrl, mv) % 
                   offsetof(DecodeCtrl, cv) % 16 == 0 && offsetof(DecodeCtrl, lred) % 16 == 0,
               "vector-loaded control arrays must be 16-byte aligned");
 
-constexpr int kSmemQ = 0;
-constexpr int kSmemRing = kSmemQ + kQBytes;
-constexpr int kSmemP = kSmemRing + kSlots * kSlotBytes;
-constexpr int kSmemCtrl = kSmemP + kPBytes;
-constexpr int kSmemBytes = kSmemCtrl + static_cast<int>(sizeof(DecodeCtrl)) + 1024;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+// Shared memory: q buffer(s) | ring | P | control. bf16: one q buffer, five
+// ring slots (HBM-bound: every slot of bytes in flight counts). FP8: two q
+// buffers, so the next segment's q is loaded and converted a whole segment
+// ahead, and four slots (the FP8 kernel is bound by its per-tile pipeline,
+// not by bytes in flight).
+template <bool kFp8>
+struct SmemLayout {
+  static constexpr int kQBufs = kFp8 ? 2 : 1;
+  static constexpr int kRing = kFp8 ? 4 : kSlots;
+  static constexpr int kQ = 0;
+  static constexpr int kRingOff = kQ + kQBufs * kQBytes;
+  static constexpr int kP = kRingOff + kRing * kSlotBytes;
+  static constexpr int kCtrl = kP + kPBytes;
+  static constexpr int kBytes = kCtrl + static_cast<int>(sizeof(DecodeCtrl)) + 1024;
+};
+static_assert(SmemLayout<false>::kBytes <= 227 * 1024 && SmemLayout<true>::kBytes <= 227 * 1024,
+              "shared memory budget");
+static_assert(SmemLayout<true>::kRing <= kSlots, "ring barriers");
 
 // TMEM column map.
 constexpr uint32_t kColS = 0;      // score buffers: bf16 cols 0-63 | 64-127; FP8 0-127 | 256-383
@@ -778,10 +790,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem + kSmemQ;
-  uint8_t* sRing = smem + kSmemRing;
-  uint8_t* sP = smem + kSmemP;
-  DecodeCtrl& c = *reinterpret_cast<DecodeCtrl*>(smem + kSmemCtrl);
+  using L = SmemLayout<kFp8>;
+  constexpr uint32_t kS = L::kRing;  // ring slots
+  uint8_t* sQ = smem + L::kQ;
+  uint8_t* sRing = smem + L::kRingOff;
+  uint8_t* sP = smem + L::kP;
+  DecodeCtrl& c = *reinterpret_cast<DecodeCtrl*>(smem + L::kCtrl);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -794,9 +808,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   // ---- setup (independent of the previous kernel's results) ----------------
   if (tid == 0) {
-    mbar_init(&c.q_full, 1);
-    mbar_init(&c.q_empty, 1);
-    for (int i = 0; i < kSlots; ++i) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&c.q_full[i], 1);
+      mbar_init(&c.q_empty[i], 1);
+      mbar_init(&c.q_conv[i], 1);
+    }
+    for (int i = 0; i < static_cast<int>(kS); ++i) {
       mbar_init(&c.slot_full[i], 1);
       mbar_init(&c.slot_empty[i], 1);
     }
@@ -811,7 +828,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     mbar_init(&c.p_full, 4 * kWG);
     mbar_init(&c.o_full, 1);
-    mbar_init(&c.q_conv, 1);
     mbar_init(&c.drain, 1);
     c.abort_flag = 0;
     c.seg_arrivals = 0;
@@ -957,8 +973,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             four_d ? kSlotBytes : static_cast<uint32_t>(nbox * rows * 128 * kBoxes);
         bool ok = true;
         for (int half = 0; half < static_cast<int>(kItemsPerTensor<kFp8>) && ok; ++half) {
-          const uint32_t slot = item % kSlots;
-          ok = warp_wait(&c.slot_empty[slot], par(item / kSlots) ^ 1u, abort_flag);
+          const uint32_t slot = item % kS;
+          ok = warp_wait(&c.slot_empty[slot], par(item / kS) ^ 1u, abort_flag);
           if (!ok) break;
           uint8_t* dst = sRing + slot * kSlotBytes;
           if (lane == 0) {
@@ -1024,7 +1040,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       first = item;
       item += kIPT;
       for (uint32_t u = 0; u < kIPT; ++u)
-        if (!warp_wait(&c.slot_full[(first + u) % kSlots], par((first + u) / kSlots), abort_flag))
+        if (!warp_wait(&c.slot_full[(first + u) % kS], par((first + u) / kS), abort_flag))
           return false;
       return true;
     };
@@ -1040,7 +1056,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           // V slot: head dims 0-127 | 128-255, each 128 token rows of 128 B
           // (MN-major A); P: 128 token rows of hi (64 B) and lo (64 B) as two
           // 64-byte-swizzled blocks 8 KB apart (one N = 128 MN-major B)
-          const uint32_t v = ring_base + (lo % kSlots) * kSlotBytes;
+          const uint32_t v = ring_base + (lo % kS) * kSlotBytes;
 #pragma unroll
           for (int kk = 0; kk < kTile / 32; ++kk)
 #pragma unroll
@@ -1049,11 +1065,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                         sw128_desc(v + r * (kSlotBytes / 2) + kk * 4096, kSlotBytes / 2, 1024),
                         sw64_desc(p_base + kk * 2048, kPBytes / 2, 512), idesc_pv,
                         (t.seg_first && kk == 0) ? 0u : 1u);
-          mma_commit(&c.slot_empty[lo % kSlots]);
+          mma_commit(&c.slot_empty[lo % kS]);
         } else {
           const uint32_t hi = lo + 1;
-          const uint32_t v_lo = ring_base + (lo % kSlots) * kSlotBytes;
-          const uint32_t v_hi = ring_base + (hi % kSlots) * kSlotBytes;
+          const uint32_t v_lo = ring_base + (lo % kS) * kSlotBytes;
+          const uint32_t v_hi = ring_base + (hi % kS) * kSlotBytes;
           // the two head-dim halves accumulate into different columns: issue
           // them alternately, so consecutive products do not wait on each other
 #pragma unroll
@@ -1065,8 +1081,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
                        sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
                        (t.seg_first && s == 0) ? 0u : 1u);
           }
-          mma_commit(&c.slot_empty[lo % kSlots]);
-          mma_commit(&c.slot_empty[hi % kSlots]);
+          mma_commit(&c.slot_empty[lo % kS]);
+          mma_commit(&c.slot_empty[hi % kS]);
         }
         mma_commit(&c.o_full);
       }
@@ -1076,9 +1092,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
     TileInfo cur, prev;
     uint32_t g = 0;
+    uint32_t qbuf = 0;  // q buffer of the current segment
     while (ok && qs.next(cur)) {
       if (cur.seg_first) {
-        ok = warp_wait(kFp8 ? &c.q_conv : &c.q_full, par(nq), abort_flag);
+        // segment nq uses q buffer nq & 1 (FP8) or the only one (bf16)
+        qbuf = kFp8 ? (nq & 1u) : 0u;
+        ok = warp_wait(kFp8 ? &c.q_conv[qbuf] : &c.q_full[0], kFp8 ? par(nq >> 1) : par(nq),
+                       abort_flag);
         ++nq;
         if (!ok) break;
       }
@@ -1093,18 +1113,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           // K slot: head dims 0-127 | 128-255 (128 token rows of 128 B, K-major);
           // q: per dims half, the 64 hi rows then the 64 lo rows (128 rows of
           // 128 B, K-major): one N = 128 operand
-          const uint32_t k = ring_base + (lo % kSlots) * kSlotBytes;
+          const uint32_t k = ring_base + (lo % kS) * kSlotBytes;
+          const uint32_t qb = q_base + qbuf * kQBytes;
 #pragma unroll
           for (int kk = 0; kk < kDim / 32; ++kk) {
             const uint32_t off = (kk >> 2) * (kSlotBytes / 2) + (kk & 3) * 32;
-            mma_f8_ss(d_s, sw128_desc(k + off, 16, 1024), sw128_desc(q_base + off, 16, 1024),
+            mma_f8_ss(d_s, sw128_desc(k + off, 16, 1024), sw128_desc(qb + off, 16, 1024),
                       idesc_qk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(&c.slot_empty[lo % kSlots]);
+          mma_commit(&c.slot_empty[lo % kS]);
         } else {
           const uint32_t hi = lo + 1;
-          const uint32_t k_lo = ring_base + (lo % kSlots) * kSlotBytes;
-          const uint32_t k_hi = ring_base + (hi % kSlots) * kSlotBytes;
+          const uint32_t k_lo = ring_base + (lo % kS) * kSlotBytes;
+          const uint32_t k_hi = ring_base + (hi % kS) * kSlotBytes;
 #pragma unroll
           for (int s = 0; s < kDim / 16; ++s) {
             const uint32_t a_addr = (s < 8 ? k_lo : k_hi) + ((s >> 2) & 1) * (kSlotBytes / 2) +
@@ -1113,11 +1134,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             mma_f16_ss(d_s, sw128_desc(a_addr, 16, 1024), sw128_desc(b_addr, 16, 1024), idesc_qk,
                        s > 0 ? 1u : 0u);
           }
-          mma_commit(&c.slot_empty[lo % kSlots]);
-          mma_commit(&c.slot_empty[hi % kSlots]);
+          mma_commit(&c.slot_empty[lo % kS]);
+          mma_commit(&c.slot_empty[hi % kS]);
         }
         mma_commit(&c.s_full[g & 1]);
-        if (cur.seg_last) mma_commit(&c.q_empty);
+        if (cur.seg_last) mma_commit(&c.q_empty[qbuf]);
       }
       __syncwarp();
       if (g >= 1 && !(ok = issue_pv(prev, g - 1))) break;
@@ -1134,28 +1155,53 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ======================= q producer =====================================
+    // ======================= q producer (FP8 cache: and publisher) ==========
+    // q of segment k goes to buffer k & 1 (FP8: the next segment's q is loaded
+    // and converted while this one runs) or the only buffer (bf16). With an
+    // FP8 cache this warp also publishes each finished segment (warp 3
+    // converts there), one segment behind: segment k - 1 after q of segment k
+    // is on its way, since k - 1's last PV is issued after k's first QK.
     const uint64_t policy = l2_policy_evict_last();
     TileStream qs, ahead;
     qs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
     ahead.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
-    TileInfo t, ta;
+    TileInfo t, ta, last;
     bool more_ahead = ahead.next(ta);  // stays one segment ahead of qs
+    bool have_last = false, ok = true;
     uint32_t k = 0;
-    while (qs.next(t)) {
-      if (!t.seg_first) continue;
-      if (!warp_wait(&c.q_empty, par(k) ^ 1u, abort_flag)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&c.q_full, kQBytes);
-        for (int r = 0; r < 4; ++r)
-          tma_load_3d(sQ + r * 8192, &tm_q, &c.q_full, r * 64, 0, t.b, policy);
+    while (ok && qs.next(t)) {
+      if (t.seg_first) {
+        const uint32_t b = kFp8 ? (k & 1u) : 0u;
+        if (!(ok = warp_wait(&c.q_empty[b], (kFp8 ? par(k >> 1) : par(k)) ^ 1u, abort_flag))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&c.q_full[b], kQBytes);
+          for (int r = 0; r < 4; ++r)
+            tma_load_3d(sQ + b * kQBytes + r * 8192, &tm_q, &c.q_full[b], r * 64, 0, t.b, policy);
+        }
+        // pull the next segment's q rows into L2 while this segment runs
+        while (more_ahead && (ta.b == t.b || !ta.seg_first)) more_ahead = ahead.next(ta);
+        if (more_ahead && lane == 0)
+          for (int r = 0; r < 4; ++r) tma_prefetch_3d(&tm_q, r * 64, 0, ta.b);
+        __syncwarp();
+        ++k;
+        if (kFp8 && have_last) {
+          if (!(ok = __all_sync(0xffffffffu,
+                                wait_count(&c.seg_arrivals, 4u * kWG * (k - 1), abort_flag))))
+            break;
+          if (lane == 0) publish_segment(p, last, c.ntot, 1u);
+          __syncwarp();
+          have_last = false;
+        }
       }
-      // pull the next segment's q rows into L2 while this segment runs
-      while (more_ahead && (ta.b == t.b || !ta.seg_first)) more_ahead = ahead.next(ta);
-      if (more_ahead && lane == 0)
-        for (int r = 0; r < 4; ++r) tma_prefetch_3d(&tm_q, r * 64, 0, ta.b);
+      if (kFp8 && t.seg_last) {
+        last = t;
+        have_last = true;
+      }
+    }
+    if (kFp8 && ok && have_last &&
+        __all_sync(0xffffffffu, wait_count(&c.seg_arrivals, 4u * kWG * k, abort_flag))) {
+      if (lane == 0) publish_segment(p, last, c.ntot, 1u);
       __syncwarp();
-      ++k;
     }
   } else if (warp == 3) {
     // ======================= FP8 converter ==================================
@@ -1173,13 +1219,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       uint32_t nq = 0;
       while (cs.next(t)) {
         if (!t.seg_first) continue;
-        if (!warp_wait(&c.q_full, par(nq), abort_flag)) break;
-        const float inv_s = q_to_e4m3(smem_u32(sQ), lane);
+        const uint32_t b = nq & 1u;  // q buffer of segment nq
+        if (!warp_wait(&c.q_full[b], par(nq >> 1), abort_flag)) break;
+        const float inv_s = q_to_e4m3(smem_u32(sQ + b * kQBytes), lane);
         if (lane == 0) c.qinv[nq & 3] = inv_s;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&c.q_conv);
+          mbar_arrive(&c.q_conv[b]);
           smem_add_release(&c.q_ready, 1u);
         }
         ++nq;
@@ -1259,11 +1306,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (!kFp8) {
-        if (lane == 0) smem_add_release(&c.seg_arrivals, 1u);
-      } else if (lane == 0 && (pt.slot >= 0 || warp == 4)) {
-        publish_segment(p, pt, c.ntot, 4u * kWG);
-      }
+      if (lane == 0) smem_add_release(&c.seg_arrivals, 1u);
       if (warp == 4 && lane == 0) MFA_TR(8, pend_g);
     };
 
@@ -1407,9 +1450,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // the tensor's one item)
       if (valid < kTile) {
         const uint32_t it = v_item<kFp8>(g, t.cta_last) + (kFp8 ? 0 : wg);
-        if (!warp_wait(&c.slot_full[it % kSlots], par(it / kSlots), abort_flag)) break;
+        if (!warp_wait(&c.slot_full[it % kS], par(it / kS), abort_flag)) break;
         if (!row_ok) {
-          const uint32_t base = smem_u32(sRing) + (it % kSlots) * kSlotBytes + row * 128 +
+          const uint32_t base = smem_u32(sRing) + (it % kS) * kSlotBytes + row * 128 +
                                 (kFp8 ? wg * (kSlotBytes / 2) : 0);
 #pragma unroll
           for (int r = 0; r < (kFp8 ? 1 : 2); ++r)
@@ -1562,7 +1605,10 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
 // ===========================================================================
 // host-side launch helper (called from mfa_api.cu)
 // ===========================================================================
-int decode_smem_bytes() { return kSmemBytes; }
+int decode_smem_bytes() {
+  return SmemLayout<false>::kBytes > SmemLayout<true>::kBytes ? SmemLayout<false>::kBytes
+                                                               : SmemLayout<true>::kBytes;
+}
 
 template <typename Kernel, typename... Args>
 static cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem,
@@ -1589,12 +1635,13 @@ static cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
     const cudaError_t err = cudaFuncSetAttribute(
-        mfa_decode_kernel<kPaged, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        mfa_decode_kernel<kPaged, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SmemLayout<kFp8>::kBytes);
     if (err != cudaSuccess) return err;
     configured_dev = dev;
   }
   return launch_pdl(mfa_decode_kernel<kPaged, kFp8>, dim3(p.grid), dim3(kDecodeThreads),
-                    kSmemBytes, stream, tq, tk, tv, p);
+                    SmemLayout<kFp8>::kBytes, stream, tq, tk, tv, p);
 }
 
 cudaError_t launch_decode(bool paged, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
