@@ -84,6 +84,58 @@ __device__ __forceinline__ void merge_latent(const float* partials, int splits, 
     }
   }
 }
+
+// The fused kernel's merge: 128 threads, thread = 4 adjacent features (16-byte
+// loads) x 2 latent rows; all splits of both rows are loaded before the first
+// add, 8 splits at a time, and summed in split order in fp32. Needs B <= 8,
+// rank a multiple of 4 and 16-byte aligned partials.
+constexpr int kMergeBatch = 8;
+__device__ __forceinline__ void merge_latent_x4(const float* partials, int splits, int B, int rank,
+                                                int m_tile0, int etid, __nv_bfloat16* latent) {
+  const int m = m_tile0 + (etid & 31) * 4;
+  const int r0 = (etid >> 5) * 2;
+  float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+  for (int s0 = 0; s0 < splits; s0 += kMergeBatch) {
+    float4 v[2][kMergeBatch];
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+        v[rr][u] = (s0 + u < splits && r0 + rr < B)
+                       ? __ldcg(reinterpret_cast<const float4*>(
+                             partials + (static_cast<int64_t>(s0 + u) * B + r0 + rr) * rank + m))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kMergeBatch; ++u)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        if (s0 + u >= splits) continue;
+        acc[rr].x += v[rr][u].x;
+        acc[rr].y += v[rr][u].y;
+        acc[rr].z += v[rr][u].z;
+        acc[rr].w += v[rr][u].w;
+      }
+  }
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int r = r0 + rr;
+    if (r >= B) break;
+    const float a[4] = {acc[rr].x, acc[rr].y, acc[rr].z, acc[rr].w};
+    __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      hi[e] = __float2bfloat16_rn(a[e]);
+      lo[e] = __float2bfloat16_rn(a[e] - __bfloat162float(hi[e]));
+    }
+    uint2 h, l;
+    h.x = static_cast<uint32_t>(__bfloat16_as_ushort(hi[0])) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi[1])) << 16);
+    h.y = static_cast<uint32_t>(__bfloat16_as_ushort(hi[2])) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi[3])) << 16);
+    l.x = static_cast<uint32_t>(__bfloat16_as_ushort(lo[0])) | (static_cast<uint32_t>(__bfloat16_as_ushort(lo[1])) << 16);
+    l.y = static_cast<uint32_t>(__bfloat16_as_ushort(lo[2])) | (static_cast<uint32_t>(__bfloat16_as_ushort(lo[3])) << 16);
+    *reinterpret_cast<uint2*>(latent + static_cast<int64_t>(2 * r) * rank + m) = h;
+    *reinterpret_cast<uint2*>(latent + static_cast<int64_t>(2 * r + 1) * rank + m) = l;
+  }
+}
 }  // namespace
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -140,22 +192,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tma_load_2d(st + kABytes / 2, &tm_w, &c.full[s], m_tile * 128 + 64, kb * 64, pol_w);
       tma_load_2d(st + kABytes, &tm_act, &c.full[s], kb * 64, 0, pol_a);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: the whole warp, one elected lane issues ----------------
     const uint32_t idesc = idesc_f16(128, n_cols, 1, 1, 0);
+    int s = 0;
+    uint32_t ph = 0;
     for (int i = 0; i < nkb; ++i) {
-      const int s = i % stages;
-      if (!mbar_wait(&c.full[s], (i / stages) & 1, abort_flag)) break;
+      if (!mbar_wait_warp(&c.full[s], ph, abort_flag)) break;
       tc_fence_after();
       const uint32_t a = smem_u32(smem + s * stage_bytes);
       const uint32_t b = a + kABytes;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        mma_f16_ss(tmem, sw128_desc(a + k * 2048, kABytes / 2, 1024), sw128_desc(b + k * 32, 16, 1024),
-                   idesc, (i > 0 || k > 0) ? 1u : 0u);
-      mma_commit(&c.empty[s]);
+        mma_f16_ss_warp(tmem, sw128_desc(a + k * 2048, kABytes / 2, 1024),
+                        sw128_desc(b + k * 32, 16, 1024), idesc, (i > 0 || k > 0) ? 1u : 0u);
+      mma_commit_warp(&c.empty[s]);
+      if (++s == stages) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
-    mma_commit(&c.acc_ready);
+    mma_commit_warp(&c.acc_ready);
   }
 
   // ---------------- epilogue: thread = output feature row ----------------
@@ -300,110 +357,135 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const uint32_t tmem = c.tmem_base;
   volatile int* abort_flag = &c.abort_flag;
 
-  if (warp == 0 && lane == 0) {
-    // ---------------- producer ----------------
+  if (warp == 0) {
+    // ---------------- producer: the whole warp, one elected lane issues ----------------
     const uint64_t pol_w = l2_policy_evict_first();
     const uint64_t pol_a = l2_policy_evict_last();
-    tma_prefetch_desc(&tm_wa);
-    tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_wb);
-    tma_prefetch_desc(&tm_lat);
-    int i = 0;
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_wa);
+      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&tm_wb);
+      tma_prefetch_desc(&tm_lat);
+    }
+    __syncwarp();
+    int s = 0;  // ring slot and phase of the next stage
+    uint32_t ph = 0;
     bool ok = true;
     if (has1) {
-      for (int kb = kb0; kb < kb1; ++kb, ++i) {
-        const int s = i % stages;
-        if (!(ok = mbar_wait(&c.empty[s], ((i / stages) & 1) ^ 1, abort_flag))) break;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!(ok = mbar_wait_warp(&c.empty[s], ph ^ 1u, abort_flag))) break;
         uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&c.full[s], kABytes + p.n1 * 128);
-        tma_load_3d(st, &tm_wa, &c.full[s], 0, kb * 64, 2 * tile1, pol_w);
-        tma_load_2d(st + kABytes, &tm_x, &c.full[s], kb * 64, 0, pol_a);
+        mbar_arrive_expect_tx_warp(&c.full[s], kABytes + p.n1 * 128);
+        tma_load_3d_warp(st, &tm_wa, &c.full[s], 0, kb * 64, 2 * tile1, pol_w);
+        tma_load_2d_warp(st + kABytes, &tm_x, &c.full[s], kb * 64, 0, pol_a);
+        if (++s == stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
     }
     if (has2 && ok) {
-      const int i2 = i;   // stage counter of the first up-projection k-block
+      int ls = s;          // slot of the next latent part
       int lat_issued = 0;  // k-blocks whose latent part is issued
       bool lat_ready = false;
       // latent parts of k-blocks [lat_issued, kb_end)
       auto issue_latent = [&](int kb_end) {
         for (; lat_issued < kb_end; ++lat_issued) {
-          const int s = (i2 + lat_issued) % stages;
-          tma_load_2d(smem + s * stage_bytes + kABytes, &tm_lat, &c.full[s], lat_issued * 64, 0,
-                      pol_a);
+          tma_load_2d_warp(smem + ls * stage_bytes + kABytes, &tm_lat, &c.full[ls],
+                           lat_issued * 64, 0, pol_a);
+          if (++ls == stages) ls = 0;
         }
       };
-      // the whole latent exists once every latent tile is merged (bounded)
+      // the whole latent exists once every latent tile is merged (bounded);
+      // every lane reads the same words, so the warp leaves the loop together
       auto await_latent = [&]() -> bool {
         volatile int* done = p.counters + kQprojDone;
         const uint64_t t0 = global_timer_ns();
+        bool good = true;
         while (*done < p.m1_tiles) {
-          if (*abort_flag) return false;
+          if (*abort_flag) {
+            good = false;
+            break;
+          }
           if (global_timer_ns() - t0 > kWaitLimitNs) {
-            record_error(6 /* MFA_ERR_TIMEOUT */);
-            *abort_flag = 1;
-            return false;
+            if (lane == 0) {
+              record_error(6 /* MFA_ERR_TIMEOUT */);
+              *abort_flag = 1;
+            }
+            good = false;
+            break;
           }
         }
+        if (!__all_sync(0xffffffffu, good)) return false;
         __threadfence();             // acquire the latent tiles
         fence_proxy_async_global();  // ... for the TMA reads that follow
         // count this CTA as having seen the latent; the last one (after all
         // latent tiles and every other reader) returns the count to zero
-        if (atomicAdd(p.counters + kQprojDone, 1) == p.m1_tiles + p.m2_tiles - 1)
+        if (lane == 0 && atomicAdd(p.counters + kQprojDone, 1) == p.m1_tiles + p.m2_tiles - 1)
           p.counters[kQprojDone] = 0;
+        __syncwarp();
         return true;
       };
-      for (int kb = 0; kb < p.k2_blocks && ok; ++kb, ++i) {
-        const int s = i % stages;
+      for (int kb = 0; kb < p.k2_blocks && ok; ++kb) {
         if (!lat_ready && kb >= stages) {
           // the ring is full of weight parts: the products need the latent now
           if (!(ok = await_latent())) break;
           lat_ready = true;
           issue_latent(kb);
         }
-        if (!(ok = mbar_wait(&c.empty[s], ((i / stages) & 1) ^ 1, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(&c.empty[s], ph ^ 1u, abort_flag))) break;
         uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&c.full[s], kABytes + p.n2 * 128);
-        tma_load_3d(st, &tm_wb, &c.full[s], 0, kb * 64, 2 * tile2, pol_w);
+        mbar_arrive_expect_tx_warp(&c.full[s], kABytes + p.n2 * 128);
+        tma_load_3d_warp(st, &tm_wb, &c.full[s], 0, kb * 64, 2 * tile2, pol_w);
         if (lat_ready) issue_latent(kb + 1);
+        if (++s == stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       if (ok && !lat_ready && await_latent()) issue_latent(p.k2_blocks);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: the whole warp, one elected lane issues ----------------
     const uint32_t idesc1 = idesc_f16(128, p.n1, 1, 1, 0);
     const uint32_t idesc2 = idesc_f16(128, p.n2, 1, 1, 0);
-    int i = 0;
+    int s = 0;
+    uint32_t ph = 0;
+    auto next = [&]() {
+      if (++s == stages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    };
     bool ok = true;
     if (has1) {
-      for (int kb = kb0; kb < kb1; ++kb, ++i) {
-        const int s = i % stages;
-        if (!(ok = mbar_wait(&c.full[s], (i / stages) & 1, abort_flag))) break;
+      for (int kb = kb0; kb < kb1; ++kb, next()) {
+        if (!(ok = mbar_wait_warp(&c.full[s], ph, abort_flag))) break;
         tc_fence_after();
         const uint32_t a = smem_u32(smem + s * stage_bytes);
         const uint32_t b = a + kABytes;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          mma_f16_ss(tmem, sw128_desc(a + k * 2048, kABytes / 2, 1024),
-                     sw128_desc(b + k * 32, 16, 1024), idesc1, (kb > kb0 || k > 0) ? 1u : 0u);
-        mma_commit(&c.empty[s]);
+          mma_f16_ss_warp(tmem, sw128_desc(a + k * 2048, kABytes / 2, 1024),
+                          sw128_desc(b + k * 32, 16, 1024), idesc1, (kb > kb0 || k > 0) ? 1u : 0u);
+        mma_commit_warp(&c.empty[s]);
       }
-      mma_commit(&c.acc1);
+      mma_commit_warp(&c.acc1);
     }
     if (has2 && ok) {
-      for (int kb = 0; kb < p.k2_blocks; ++kb, ++i) {
-        const int s = i % stages;
-        if (!mbar_wait(&c.full[s], (i / stages) & 1, abort_flag)) break;
+      for (int kb = 0; kb < p.k2_blocks; ++kb, next()) {
+        if (!mbar_wait_warp(&c.full[s], ph, abort_flag)) break;
         tc_fence_after();
         const uint32_t a = smem_u32(smem + s * stage_bytes);
         const uint32_t b = a + kABytes;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          mma_f16_ss(tmem + 32, sw128_desc(a + k * 2048, kABytes / 2, 1024),
-                     sw128_desc(b + k * 32, 16, 1024), idesc2, (kb > 0 || k > 0) ? 1u : 0u);
-        mma_commit(&c.empty[s]);
+          mma_f16_ss_warp(tmem + 32, sw128_desc(a + k * 2048, kABytes / 2, 1024),
+                          sw128_desc(b + k * 32, 16, 1024), idesc2, (kb > 0 || k > 0) ? 1u : 0u);
+        mma_commit_warp(&c.empty[s]);
       }
     }
-    if (has2) mma_commit(&c.acc2);
+    if (has2) mma_commit_warp(&c.acc2);
   }
   __syncwarp();
 
@@ -438,7 +520,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     epi_sync();
     if (c.is_last) {
       __threadfence();
-      merge_latent<4>(p.partials, p.splits, B, p.rank, m, p.latent);
+      merge_latent_x4(p.partials, p.splits, B, p.rank, tile1 * 128, etid, p.latent);
       __threadfence();
       epi_sync();
       if (etid == 0) {
