@@ -94,6 +94,7 @@ struct __align__(16) DecodeCtrl {
   unsigned seg_arrivals;  // bf16 cache: softmax-warp arrivals at segment ends (never wraps)
   unsigned q_ready;       // FP8 cache: segments whose q is converted (never wraps)
   float qinv[4];          // FP8 cache: score scale 1/s of segment k at [k & 3]
+  unsigned qmax[16];      // FP8 cache: per-warp max |q| bits of the first segment's group conversion
   int b_start, off_start, tiles;
   int scan_warp[kDecodeThreads / 32];
   int lens[kDecodeThreads];  // validated seq_lens when batch <= kDecodeThreads
@@ -170,11 +171,6 @@ __device__ __forceinline__ int valid_len(const DecodeParams& p, int b) {
 }
 
 // All lanes wait; the outcome is made warp-uniform.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
-  return __all_sync(0xffffffffu, ok);
-}
-
 __device__ __forceinline__ uint32_t par(uint32_t u) { return u & 1u; }
 
 // ---------------------------------------------------------------------------
@@ -605,50 +601,129 @@ __device__ __forceinline__ float q_max_abs(uint32_t base, int lane) {
   return __uint_as_float(top << 16);
 }
 
-__device__ __forceinline__ float q_to_e4m3(uint32_t base, int lane) {
-  // s = 2^(7 - E) with max|q| in [2^E, 2^(E+1)); the exponent field is clamped
-  // so that s and 1/s stay normal floats (an all-zero q takes any scale)
-  int ebits = static_cast<int>((__float_as_uint(q_max_abs(base, lane)) >> 23) & 0xFF);
+// Score scale of a q whose largest |element| has the bf16 bits `top`:
+// s = 2^(7 - E) with max|q| in [2^E, 2^(E+1)); the exponent field is clamped
+// so that s and 1/s stay normal floats (an all-zero q takes any scale).
+__device__ __forceinline__ void q_scale(uint32_t top, float& s, float& inv_s) {
+  int ebits = static_cast<int>(((top << 16) >> 23) & 0xFF);
   ebits = ebits < 8 ? 8 : (ebits > 253 ? 253 : ebits);
-  const float s = __uint_as_float(static_cast<uint32_t>(261 - ebits) << 23);
-  const float inv_s = __uint_as_float(static_cast<uint32_t>(ebits - 7) << 23);
+  s = __uint_as_float(static_cast<uint32_t>(261 - ebits) << 23);
+  inv_s = __uint_as_float(static_cast<uint32_t>(ebits - 7) << 23);
+}
+
+// The conversion works on units of 16 dims of one head and dims half: 32 bytes
+// of bf16 q in, 16 bytes of hi and 16 bytes of lo E4M3 out. The loaded q of a
+// head and dims half is two 128-byte rows (dims 0-63 | 64-127 of the half,
+// 8 KB apart, 16-byte chunks swizzled by the head); its E4M3 pair takes the
+// same two rows, hi then lo. Unit m (0-7) reads chunks 2m, 2m+1 of that span
+// and writes chunk m of each row, so a head's units are converted only after
+// all eight have read their input. A thread takes four consecutive units (one
+// row half) and holds their input in registers; the code is one short rolled
+// loop: it runs once per segment, where a long unrolled body would mostly wait
+// for instruction fetch.
+constexpr int kQUnits = 2 * kHeads * 8;  // head x dims half x 16-dim unit
+constexpr int kQUnitsPerThread = 4;
+
+// Loads the input of units [4 t, 4 t + 4): head h = t / 4, dims half c = (t / 2) & 1,
+// units 4 (t & 1) .. + 3 (input row k = t & 1).
+__device__ __forceinline__ void q_load_units(uint32_t base, int t, uint4 (&in)[8]) {
+  const int h = t >> 2, c = (t >> 1) & 1, k = t & 1, sw = h & 7;
+  const uint32_t row = base + (2 * c + k) * 8192 + h * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) in[j] = ld_shared_v4(row + ((j ^ sw) << 4));
+}
+
+__device__ __forceinline__ uint32_t q_units_max(const uint4 (&in)[8]) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    m = __vmaxu2(m, __vmaxu2(__vmaxu2(in[j].x & 0x7FFF7FFFu, in[j].y & 0x7FFF7FFFu),
+                             __vmaxu2(in[j].z & 0x7FFF7FFFu, in[j].w & 0x7FFF7FFFu)));
+  return m;
+}
+
+// Writes the E4M3 pairs of the units loaded by q_load_units(base, t, in).
+__device__ __forceinline__ void q_store_units(uint32_t base, int t, float s, uint4 (&in)[8]) {
+  const int h = t >> 2, c = (t >> 1) & 1, sw = h & 7;
+  const uint32_t hi_row = base + c * 16384 + h * 128;
+  const uint32_t lo_row = hi_row + 8192;
 #pragma unroll 1
-  for (int h = lane; h < kHeads; h += 32) {
-    const int sw = h & 7;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      // the whole row of this head and dims half first: the outputs land on it
-      uint4 in[16];
+  for (int q = 0; q < kQUnitsPerThread; ++q) {
+    const int m = 4 * (t & 1) + q;  // output chunk: dims 16m..16m+15 of the half
+    uint32_t w[8];
 #pragma unroll
-      for (int k = 0; k < 2; ++k)
+    for (int u = 0; u < 2; ++u) {
+      const uint4 v = in[u];
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          in[8 * k + j] = ld_shared_v4(base + (2 * c + k) * 8192 + h * 128 + ((j ^ sw) << 4));
-      const uint32_t hi_row = base + c * 16384 + h * 128;
-      const uint32_t lo_row = hi_row + 8192;
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {  // output chunk m: dims 16m..16m+15 of the half
-        uint32_t w[8];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint4 v = in[2 * m + u];
-          const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            // four bf16 -> two hi/lo pairs
-            const uint32_t p0 = split_e4m3x2(__uint_as_float(wd[e] << 16) * s,
-                                             __uint_as_float(wd[e] & 0xFFFF0000u) * s);
-            const uint32_t p1 = split_e4m3x2(__uint_as_float(wd[e + 1] << 16) * s,
-                                             __uint_as_float(wd[e + 1] & 0xFFFF0000u) * s);
-            w[4 * u + e / 2] = (p0 & 0xFFFFu) | (p1 << 16);          // hi bytes
-            w[4 * u + 2 + e / 2] = (p0 >> 16) | (p1 & 0xFFFF0000u);  // lo bytes
-          }
-        }
-        st_shared_v4(hi_row + ((m ^ sw) << 4), w[0], w[1], w[4], w[5]);
-        st_shared_v4(lo_row + ((m ^ sw) << 4), w[2], w[3], w[6], w[7]);
+      for (int e = 0; e < 4; e += 2) {
+        // four bf16 -> two hi/lo pairs
+        const uint32_t p0 = split_e4m3x2(__uint_as_float(wd[e] << 16) * s,
+                                         __uint_as_float(wd[e] & 0xFFFF0000u) * s);
+        const uint32_t p1 = split_e4m3x2(__uint_as_float(wd[e + 1] << 16) * s,
+                                         __uint_as_float(wd[e + 1] & 0xFFFF0000u) * s);
+        w[4 * u + e / 2] = (p0 & 0xFFFFu) | (p1 << 16);          // hi bytes
+        w[4 * u + 2 + e / 2] = (p0 >> 16) | (p1 & 0xFFFF0000u);  // lo bytes
       }
     }
+    st_shared_v4(hi_row + ((m ^ sw) << 4), w[0], w[1], w[4], w[5]);
+    st_shared_v4(lo_row + ((m ^ sw) << 4), w[2], w[3], w[6], w[7]);
+#pragma unroll
+    for (int j = 0; j < 6; ++j) in[j] = in[j + 2];  // next unit's input to in[0..1]
   }
+}
+
+// q of a segment to its exact E4M3 pair, in place, by one warp; returns 1/s.
+__device__ __forceinline__ float q_to_e4m3(uint32_t base, int lane) {
+  float s, inv_s;
+  q_scale(__float_as_uint(q_max_abs(base, lane)) >> 16, s, inv_s);
+  // rounds of 32 threads x 4 units = 16 whole (head, dims half) spans
+#pragma unroll 1
+  for (int r = 0; r < kQUnits / (32 * kQUnitsPerThread); ++r) {
+    uint4 in[8];
+    const int t = r * 32 + lane;
+    q_load_units(base, t, in);
+    __syncwarp();  // both halves of each span read before either writes
+    q_store_units(base, t, s, in);
+  }
+  return inv_s;
+}
+
+// The same conversion by warp 3 and the softmax warps together, for a CTA's
+// first segment (its first product waits for it, and the softmax warps would
+// otherwise wait for that product). gtid = thread index - 96; threads below
+// kQUnits / 4 take four units each. Every thread of the group calls it exactly
+// once, also after a failed wait (work = false): it holds two barriers
+// (named barrier 1) of the whole group, the first of which also orders every
+// read of q before the in-place writes. The softmax warps only arrive at the
+// second; warp 3 waits there, then publishes.
+constexpr int kQGroupWarps = 1 + 4 * kWG;
+constexpr int kQGroupThreads = 32 * kQGroupWarps;
+static_assert(kQGroupThreads * kQUnitsPerThread >= kQUnits, "group covers q in one round");
+__device__ __forceinline__ float q_to_e4m3_group(uint32_t base, int gtid, bool work, bool publisher,
+                                                 unsigned* part) {
+  const bool mine = work && gtid < kQUnits / kQUnitsPerThread;
+  uint4 in[8];
+  uint32_t m = 0;
+  if (mine) {
+    q_load_units(base, gtid, in);
+    m = q_units_max(in);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = __vmaxu2(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((gtid & 31) == 0) part[gtid >> 5] = (m >> 16) > (m & 0xFFFFu) ? (m >> 16) : (m & 0xFFFFu);
+  asm volatile("bar.sync 1, %0;" ::"n"(kQGroupThreads) : "memory");
+  uint32_t top = 0;
+#pragma unroll
+  for (int w = 0; w < kQGroupWarps; ++w) top = part[w] > top ? part[w] : top;
+  float s, inv_s;
+  q_scale(top, s, inv_s);
+  if (mine) q_store_units(base, gtid, s, in);
+  fence_proxy_async_smem();
+  if (publisher)
+    asm volatile("bar.sync 1, %0;" ::"n"(kQGroupThreads) : "memory");
+  else
+    asm volatile("bar.arrive 1, %0;" ::"n"(kQGroupThreads) : "memory");
   return inv_s;
 }
 
@@ -974,7 +1049,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         bool ok = true;
         for (int half = 0; half < static_cast<int>(kItemsPerTensor<kFp8>) && ok; ++half) {
           const uint32_t slot = item % kS;
-          ok = warp_wait(&c.slot_empty[slot], par(item / kS) ^ 1u, abort_flag);
+          ok = mbar_wait_warp(&c.slot_empty[slot], par(item / kS) ^ 1u, abort_flag);
           if (!ok) break;
           uint8_t* dst = sRing + slot * kSlotBytes;
           if (lane == 0) {
@@ -1040,53 +1115,53 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       first = item;
       item += kIPT;
       for (uint32_t u = 0; u < kIPT; ++u)
-        if (!warp_wait(&c.slot_full[(first + u) % kS], par((first + u) / kS), abort_flag))
+        if (!mbar_wait_warp(&c.slot_full[(first + u) % kS], par((first + u) / kS), abort_flag))
           return false;
       return true;
     };
 
     auto issue_pv = [&](const TileInfo& t, uint32_t j) -> bool {
-      if (!warp_wait(&c.p_full, par(j), abort_flag)) return false;
+      if (!mbar_wait_warp(&c.p_full, par(j), abort_flag)) return false;
       uint32_t lo;
       if (!take_items(lo)) return false;
       tc_fence_after();
-      if (lane == 0) {
-        MFA_TR(3, j);
-        if (kFp8) {
-          // V slot: head dims 0-127 | 128-255, each 128 token rows of 128 B
-          // (MN-major A); P: 128 token rows of hi (64 B) and lo (64 B) as two
-          // 64-byte-swizzled blocks 8 KB apart (one N = 128 MN-major B)
-          const uint32_t v = ring_base + (lo % kS) * kSlotBytes;
+      if (lane == 0) MFA_TR(3, j);
+      // the whole warp issues (one elected lane; see mma_f16_ss_warp)
+      if (kFp8) {
+        // V slot: head dims 0-127 | 128-255, each 128 token rows of 128 B
+        // (MN-major A); P: 128 token rows of hi (64 B) and lo (64 B) as two
+        // 64-byte-swizzled blocks 8 KB apart (one N = 128 MN-major B)
+        const uint32_t v = ring_base + (lo % kS) * kSlotBytes;
 #pragma unroll
-          for (int kk = 0; kk < kTile / 32; ++kk)
+        for (int kk = 0; kk < kTile / 32; ++kk)
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
-              mma_f8_ss(tmem + o_base<kFp8>(t.seg, r),
-                        sw128_desc(v + r * (kSlotBytes / 2) + kk * 4096, kSlotBytes / 2, 1024),
-                        sw64_desc(p_base + kk * 2048, kPBytes / 2, 512), idesc_pv,
-                        (t.seg_first && kk == 0) ? 0u : 1u);
-          mma_commit(&c.slot_empty[lo % kS]);
-        } else {
-          const uint32_t hi = lo + 1;
-          const uint32_t v_lo = ring_base + (lo % kS) * kSlotBytes;
-          const uint32_t v_hi = ring_base + (hi % kS) * kSlotBytes;
-          // the two head-dim halves accumulate into different columns: issue
-          // them alternately, so consecutive products do not wait on each other
+          for (int r = 0; r < 2; ++r)
+            mma_f8_ss_warp(tmem + o_base<kFp8>(t.seg, r),
+                           sw128_desc(v + r * (kSlotBytes / 2) + kk * 4096, kSlotBytes / 2, 1024),
+                           sw64_desc(p_base + kk * 2048, kPBytes / 2, 512), idesc_pv,
+                           (t.seg_first && kk == 0) ? 0u : 1u);
+        mma_commit_warp(&c.slot_empty[lo % kS]);
+      } else {
+        const uint32_t hi = lo + 1;
+        const uint32_t v_lo = ring_base + (lo % kS) * kSlotBytes;
+        const uint32_t v_hi = ring_base + (hi % kS) * kSlotBytes;
+        // the two head-dim halves accumulate into different columns: issue
+        // them alternately, so consecutive products do not wait on each other
 #pragma unroll
-          for (int s = 0; s < kTile / 16; ++s) {
-            mma_f16_ss(tmem + o_base<kFp8>(t.seg, 0), sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
-                       sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
-                       (t.seg_first && s == 0) ? 0u : 1u);
-            mma_f16_ss(tmem + o_base<kFp8>(t.seg, 1), sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
-                       sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
-                       (t.seg_first && s == 0) ? 0u : 1u);
-          }
-          mma_commit(&c.slot_empty[lo % kS]);
-          mma_commit(&c.slot_empty[hi % kS]);
+        for (int s = 0; s < kTile / 16; ++s) {
+          mma_f16_ss_warp(tmem + o_base<kFp8>(t.seg, 0),
+                          sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
+                          sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                          (t.seg_first && s == 0) ? 0u : 1u);
+          mma_f16_ss_warp(tmem + o_base<kFp8>(t.seg, 1),
+                          sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
+                          sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                          (t.seg_first && s == 0) ? 0u : 1u);
         }
-        mma_commit(&c.o_full);
+        mma_commit_warp(&c.slot_empty[lo % kS]);
+        mma_commit_warp(&c.slot_empty[hi % kS]);
       }
-      __syncwarp();
+      mma_commit_warp(&c.o_full);
       return true;
     };
 
@@ -1097,50 +1172,47 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (cur.seg_first) {
         // segment nq uses q buffer nq & 1 (FP8) or the only one (bf16)
         qbuf = kFp8 ? (nq & 1u) : 0u;
-        ok = warp_wait(kFp8 ? &c.q_conv[qbuf] : &c.q_full[0], kFp8 ? par(nq >> 1) : par(nq),
+        ok = mbar_wait_warp(kFp8 ? &c.q_conv[qbuf] : &c.q_full[0], kFp8 ? par(nq >> 1) : par(nq),
                        abort_flag);
         ++nq;
         if (!ok) break;
       }
-      if (g >= 2 && !(ok = warp_wait(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag))) break;
+      if (g >= 2 && !(ok = mbar_wait_warp(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag))) break;
       uint32_t lo;
       if (!(ok = take_items(lo))) break;
       tc_fence_after();
-      if (lane == 0) {
-        MFA_TR(2, g);
-        const uint32_t d_s = tmem + s_cols<kFp8>(g);
-        if (kFp8) {
-          // K slot: head dims 0-127 | 128-255 (128 token rows of 128 B, K-major);
-          // q: per dims half, the 64 hi rows then the 64 lo rows (128 rows of
-          // 128 B, K-major): one N = 128 operand
-          const uint32_t k = ring_base + (lo % kS) * kSlotBytes;
-          const uint32_t qb = q_base + qbuf * kQBytes;
+      if (lane == 0) MFA_TR(2, g);
+      const uint32_t d_s = tmem + s_cols<kFp8>(g);
+      if (kFp8) {
+        // K slot: head dims 0-127 | 128-255 (128 token rows of 128 B, K-major);
+        // q: per dims half, the 64 hi rows then the 64 lo rows (128 rows of
+        // 128 B, K-major): one N = 128 operand
+        const uint32_t k = ring_base + (lo % kS) * kSlotBytes;
+        const uint32_t qb = q_base + qbuf * kQBytes;
 #pragma unroll
-          for (int kk = 0; kk < kDim / 32; ++kk) {
-            const uint32_t off = (kk >> 2) * (kSlotBytes / 2) + (kk & 3) * 32;
-            mma_f8_ss(d_s, sw128_desc(k + off, 16, 1024), sw128_desc(qb + off, 16, 1024),
-                      idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&c.slot_empty[lo % kS]);
-        } else {
-          const uint32_t hi = lo + 1;
-          const uint32_t k_lo = ring_base + (lo % kS) * kSlotBytes;
-          const uint32_t k_hi = ring_base + (hi % kS) * kSlotBytes;
-#pragma unroll
-          for (int s = 0; s < kDim / 16; ++s) {
-            const uint32_t a_addr = (s < 8 ? k_lo : k_hi) + ((s >> 2) & 1) * (kSlotBytes / 2) +
-                                    (s & 3) * 32;
-            const uint32_t b_addr = q_base + (s >> 2) * 8192 + (s & 3) * 32;
-            mma_f16_ss(d_s, sw128_desc(a_addr, 16, 1024), sw128_desc(b_addr, 16, 1024), idesc_qk,
-                       s > 0 ? 1u : 0u);
-          }
-          mma_commit(&c.slot_empty[lo % kS]);
-          mma_commit(&c.slot_empty[hi % kS]);
+        for (int kk = 0; kk < kDim / 32; ++kk) {
+          const uint32_t off = (kk >> 2) * (kSlotBytes / 2) + (kk & 3) * 32;
+          mma_f8_ss_warp(d_s, sw128_desc(k + off, 16, 1024), sw128_desc(qb + off, 16, 1024),
+                         idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&c.s_full[g & 1]);
-        if (cur.seg_last) mma_commit(&c.q_empty[qbuf]);
+        mma_commit_warp(&c.slot_empty[lo % kS]);
+      } else {
+        const uint32_t hi = lo + 1;
+        const uint32_t k_lo = ring_base + (lo % kS) * kSlotBytes;
+        const uint32_t k_hi = ring_base + (hi % kS) * kSlotBytes;
+#pragma unroll
+        for (int s = 0; s < kDim / 16; ++s) {
+          const uint32_t a_addr = (s < 8 ? k_lo : k_hi) + ((s >> 2) & 1) * (kSlotBytes / 2) +
+                                  (s & 3) * 32;
+          const uint32_t b_addr = q_base + (s >> 2) * 8192 + (s & 3) * 32;
+          mma_f16_ss_warp(d_s, sw128_desc(a_addr, 16, 1024), sw128_desc(b_addr, 16, 1024),
+                          idesc_qk, s > 0 ? 1u : 0u);
+        }
+        mma_commit_warp(&c.slot_empty[lo % kS]);
+        mma_commit_warp(&c.slot_empty[hi % kS]);
       }
-      __syncwarp();
+      mma_commit_warp(&c.s_full[g & 1]);
+      if (cur.seg_last) mma_commit_warp(&c.q_empty[qbuf]);
       if (g >= 1 && !(ok = issue_pv(prev, g - 1))) break;
       prev = cur;
       ++g;
@@ -1172,7 +1244,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     while (ok && qs.next(t)) {
       if (t.seg_first) {
         const uint32_t b = kFp8 ? (k & 1u) : 0u;
-        if (!(ok = warp_wait(&c.q_empty[b], (kFp8 ? par(k >> 1) : par(k)) ^ 1u, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(&c.q_empty[b], (kFp8 ? par(k >> 1) : par(k)) ^ 1u, abort_flag))) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(&c.q_full[b], kQBytes);
           for (int r = 0; r < 4; ++r)
@@ -1220,8 +1292,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       while (cs.next(t)) {
         if (!t.seg_first) continue;
         const uint32_t b = nq & 1u;  // q buffer of segment nq
-        if (!warp_wait(&c.q_full[b], par(nq >> 1), abort_flag)) break;
-        const float inv_s = q_to_e4m3(smem_u32(sQ + b * kQBytes), lane);
+        const bool got = mbar_wait_warp(&c.q_full[b], par(nq >> 1), abort_flag);
+        // the first segment with the softmax warps (they call the same function)
+        const float inv_s = nq == 0 ? q_to_e4m3_group(smem_u32(sQ), tid - 96, got, true, c.qmax)
+                            : got   ? q_to_e4m3(smem_u32(sQ + b * kQBytes), lane)
+                                    : 0.f;
+        if (!got) break;
         if (lane == 0) c.qinv[nq & 3] = inv_s;
         fence_proxy_async_smem();
         __syncwarp();
@@ -1256,6 +1332,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
     TileStream ts;
     ts.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    if (kFp8) {
+      // the first segment's q conversion, with warp 3 (which publishes it)
+      TileStream first = ts;
+      TileInfo tf;
+      if (first.next(tf)) {
+        const bool got = mbar_wait_warp(&c.q_full[0], 0u, abort_flag);
+        q_to_e4m3_group(smem_u32(sQ), tid - 96, got, false, c.qmax);
+      }
+    }
     TileInfo t;
     uint32_t g = 0, nseg = 0;
     float m_run = -INFINITY;  // running max in use (log2 units), head hbase + lane
@@ -1321,7 +1406,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
       }
       // ---- scores of this tile (this warpgroup's 32 heads) ---------------
-      if (!warp_wait(&c.s_full[g & 1], par(g >> 1), abort_flag)) break;
+      if (!mbar_wait_warp(&c.s_full[g & 1], par(g >> 1), abort_flag)) break;
       if (warp == 4 && lane == 0) MFA_TR(4, g);
       tc_fence_after();
       float s[kWGHeads];
@@ -1358,7 +1443,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.red_full[wg][g & 1]);
-      if (!warp_wait(&c.red_full[wg][g & 1], par(g >> 1), abort_flag)) break;
+      if (!mbar_wait_warp(&c.red_full[wg][g & 1], par(g >> 1), abort_flag)) break;
       if (warp == 4 && lane == 0) MFA_TR(5, g);
       const float tmax = fmaxf(fmaxf(c.red[g & 1][wg][0][lane], c.red[g & 1][wg][1][lane]),
                                fmaxf(c.red[g & 1][wg][2][lane], c.red[g & 1][wg][3][lane]));
@@ -1408,7 +1493,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
       // ---- P buffer and O are free once the previous tile's PV completed --
       if (warp == 4 && lane == 0) MFA_TR(6, g);
-      if (g >= 1 && !warp_wait(&c.o_full, par(g - 1), abort_flag)) break;
+      if (g >= 1 && !mbar_wait_warp(&c.o_full, par(g - 1), abort_flag)) break;
       tc_fence_after();
       if (rescale && !t.seg_first) {
 #pragma unroll 1
@@ -1450,7 +1535,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // the tensor's one item)
       if (valid < kTile) {
         const uint32_t it = v_item<kFp8>(g, t.cta_last) + (kFp8 ? 0 : wg);
-        if (!warp_wait(&c.slot_full[it % kS], par(it / kS), abort_flag)) break;
+        if (!mbar_wait_warp(&c.slot_full[it % kS], par(it / kS), abort_flag)) break;
         if (!row_ok) {
           const uint32_t base = smem_u32(sRing) + (it % kS) * kSlotBytes + row * 128 +
                                 (kFp8 ? wg * (kSlotBytes / 2) : 0);
@@ -1486,7 +1571,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&c.l_full[wg]);
-        if (!warp_wait(&c.l_full[wg], par(nseg), abort_flag)) break;
+        if (!mbar_wait_warp(&c.l_full[wg], par(nseg), abort_flag)) break;
         const float l = c.lred[wg][0][lane] + c.lred[wg][1][lane] + c.lred[wg][2][lane] +
                         c.lred[wg][3][lane];
         // the next tile starts a new segment: the row sums restart from zero
@@ -1507,7 +1592,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         have_pending = true;
         if (kFp8 && !t.cta_last) {
           // single O buffer: read out now, before the next segment's first PV
-          if (!warp_wait(&c.o_full, par(g), abort_flag)) break;
+          if (!mbar_wait_warp(&c.o_full, par(g), abort_flag)) break;
           tc_fence_after();
           write_segment(pend);
           have_pending = false;
@@ -1516,7 +1601,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       ++g;
     }
     // the CTA's last segment: after its last PV
-    if (have_pending && !*abort_flag && warp_wait(&c.o_full, par(g - 1), abort_flag)) {
+    if (have_pending && !*abort_flag && mbar_wait_warp(&c.o_full, par(g - 1), abort_flag)) {
       tc_fence_after();
       write_segment(pend);
     }
