@@ -412,13 +412,22 @@ __device__ __forceinline__ void publish_segment(const DecodeParams& p, const Til
                                                 long long ntot, unsigned arrivals) {
   unsigned long long word = kReadyNone;
   if (t.slot >= 0) {
-    __threadfence();  // the partial (made visible to this thread) before the arrival
+    // one acquire-release increment: its release half orders this segment's
+    // partial (whose stores this thread has acquired) before the arrival, its
+    // acquire half the other arrivers' partials before what follows; wraps
+    // to 0 on the last arrival
     const unsigned n = arrivals * static_cast<unsigned>(segments_of(p, t, ntot));
-    if (atomicInc(p.ws_arrive + t.b, n - 1) != n - 1) return;  // wraps to 0 on the last
-    __threadfence();  // the other arrivers' partials before the ready words
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p.ws_arrive + t.b), "r"(n - 1)
+                 : "memory");
+    if (old != n - 1) return;
     word = kReadyMerge | (static_cast<unsigned long long>(t.gtile - t.tile) << 2) |
            (static_cast<unsigned long long>(ntot) << 32);
   }
+  // release: everything this thread has observed before the ready words
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
   st_ready4(p.ws_ready + 4 * static_cast<int64_t>(t.b), word);
 }
 
@@ -731,22 +740,26 @@ constexpr int kCombineHeads = 16;  // heads per CTA
 constexpr int kCombineDims = 16;   // head-dim elements per thread (kDim / 16 threads per head)
 constexpr int kCombineBatch = 4;   // partials loaded per round trip
 
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* w) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+  return v;
+}
+
 // Waits (bounded) until *w is non-zero; returns it, or 0 after the wait limit.
-// Polls with plain volatile loads; the fence after the last one makes it an
-// acquire, ordering the caller's reads of the partials after the word.
+// Polls with acquire loads, ordering the caller's reads of the partials after
+// the word.
 __device__ unsigned long long wait_ready(const unsigned long long* w) {
-  const volatile unsigned long long* vw = w;
-  unsigned long long v = *vw;
+  unsigned long long v = ld_acquire_u64(w);
   if (v == 0) {
     const uint64_t t0 = global_timer_ns();
-    while ((v = *vw) == 0) {
+    while ((v = ld_acquire_u64(w)) == 0) {
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         record_error(6 /* MFA_ERR_TIMEOUT */);
         return 0;
       }
     }
   }
-  __threadfence();
   return v;
 }
 
