@@ -129,7 +129,7 @@ static_assert(SmemLayout<false>::kBytes <= 227 * 1024 && SmemLayout<true>::kByte
 static_assert(SmemLayout<true>::kRing <= kSlots, "ring barriers");
 
 // TMEM column map.
-constexpr uint32_t kColS = 0;      // score buffers: bf16 cols 0-63 | 64-127; FP8 0-127 | 256-383
+constexpr uint32_t kColS = 0;      // score buffers: bf16 cols 0-63 | 64-127; FP8 0-63 | 256-319
 constexpr uint32_t kColOlo = 128;  // O^T rows 0..127
 constexpr uint32_t kColOhi = 192;  // O^T rows 128..255
 constexpr uint32_t kColObuf = 256; // column offset of the odd segments' O pair
@@ -147,9 +147,10 @@ __device__ __forceinline__ uint32_t o_base(int seg, int r) {
   return kFp8 ? (r ? 384u : 128u) : o_cols(seg) + (r ? kColOhi : kColOlo);
 }
 
-// Score buffer of tile g. bf16: 64 columns (heads). FP8: 128 columns, K.q_hi
-// in 0-63 and K.q_lo in 64-127 (one N = 128 product per step reads each K
-// step once for both parts).
+// Score buffer of tile g: 64 columns (heads). With an FP8 cache the products
+// with q's hi and lo parts accumulate into the same columns (two N = 64
+// products per step): the tensor core adds the parts, not the softmax warps,
+// whose instruction count bounds the FP8 tile rate.
 template <bool kFp8>
 __device__ __forceinline__ uint32_t s_cols(uint32_t g) {
   return kColS + (g & 1) * (kFp8 ? 256u : 64u);
@@ -1113,7 +1114,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // bf16 cache: kind::f16 products of bf16 operands. FP8 cache: kind::f8f6f4
     // products of E4M3 operands straight from the ring (K, V), with q and P
     // each given as an exact E4M3 pair hi + lo (two products per step).
-    constexpr uint32_t idesc_qk = idesc_f16(128, kFp8 ? 128 : 64, kFp8 ? 0 : 1, 0, 0);
+    constexpr uint32_t idesc_qk = idesc_f16(128, 64, kFp8 ? 0 : 1, 0, 0);
     constexpr uint32_t idesc_pv = idesc_f16(128, kFp8 ? 128 : 64, kFp8 ? 0 : 1, 1, 1);
     constexpr uint32_t kIPT = kItemsPerTensor<kFp8>;
     const uint32_t q_base = smem_u32(sQ);
@@ -1198,15 +1199,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       const uint32_t d_s = tmem + s_cols<kFp8>(g);
       if (kFp8) {
         // K slot: head dims 0-127 | 128-255 (128 token rows of 128 B, K-major);
-        // q: per dims half, the 64 hi rows then the 64 lo rows (128 rows of
-        // 128 B, K-major): one N = 128 operand
+        // q: per dims half, the 64 hi rows then the 64 lo rows (128 B each,
+        // K-major): two N = 64 operands, both accumulated into S
         const uint32_t k = ring_base + (lo % kS) * kSlotBytes;
         const uint32_t qb = q_base + qbuf * kQBytes;
 #pragma unroll
         for (int kk = 0; kk < kDim / 32; ++kk) {
           const uint32_t off = (kk >> 2) * (kSlotBytes / 2) + (kk & 3) * 32;
-          mma_f8_ss_warp(d_s, sw128_desc(k + off, 16, 1024), sw128_desc(qb + off, 16, 1024),
-                         idesc_qk, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int part = 0; part < 2; ++part)
+            mma_f8_ss_warp(d_s, sw128_desc(k + off, 16, 1024),
+                           sw128_desc(qb + off + part * (kQBytes / 4), 16, 1024), idesc_qk,
+                           (kk > 0 || part > 0) ? 1u : 0u);
         }
         mma_commit_warp(&c.slot_empty[lo % kS]);
       } else {
@@ -1422,21 +1426,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (!mbar_wait_warp(&c.s_full[g & 1], par(g >> 1), abort_flag)) break;
       if (warp == 4 && lane == 0) MFA_TR(4, g);
       tc_fence_after();
+      // scaled scores (log2 units); the maximum's own term is then exactly 0
       float s[kWGHeads];
       {
         uint32_t r[32];
         tmem_ld32(tmem + lane_addr + s_cols<kFp8>(g) + hbase, r);
-        if (kFp8) {
-          uint32_t r2[32];
-          tmem_ld32(tmem + lane_addr + s_cols<kFp8>(g) + 64 + hbase, r2);
-          tmem_wait_ld();
+        tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]) + __uint_as_float(r2[h]);
-        } else {
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]);
-        }
+        for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]) * sl2_seg;
       }
       tc_fence_before();
       __syncwarp();
@@ -1444,8 +1441,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
       const int valid = min(kTile, t.L - t.tile * kTile);
       const bool row_ok = row < valid;
+      if (valid < kTile && !row_ok) {  // rows past the end: no weight
 #pragma unroll
-      for (int h = 0; h < kWGHeads; ++h) s[h] = row_ok ? s[h] * sl2_seg : -INFINITY;
+        for (int h = 0; h < kWGHeads; ++h) s[h] = -INFINITY;
+      }
 
       // ---- per-head maximum over the tile's 128 rows --------------------
       {
