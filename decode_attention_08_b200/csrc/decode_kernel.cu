@@ -1696,7 +1696,12 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
   // back to zero for the next call, which sets it only after this kernel
   // has completed
   if (nt > 0 && threadIdx.x == 0 && word != 0) *ready = 0;
-  griddep_wait();
+  // One block waits for the attention grid to complete, so this grid never
+  // completes before it: a later kernel that waits for this one (the next
+  // call) also waits for the attention kernel. The other blocks leave as soon
+  // as their sequence is merged, so the blocks that did not fit beside the
+  // attention CTAs (large batches) start without waiting for that grid's end.
+  if (blockIdx.x == 0 && blockIdx.y == 0) griddep_wait();
 }
 
 // ===========================================================================
