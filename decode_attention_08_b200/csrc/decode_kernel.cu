@@ -514,13 +514,6 @@ __device__ void balanced_plan(const DecodeParams& p, DecodeCtrl& c, const int* l
   __syncthreads();
 }
 
-__device__ __forceinline__ void store_out(const DecodeParams& p, int b, int h, int d, float v) {
-  if (p.out_f32)
-    static_cast<float*>(p.out)[b * p.out_sb + h * p.out_sh + d] = v;
-  else
-    static_cast<__nv_bfloat16*>(p.out)[b * p.out_sb + h * p.out_sh + d] = __float2bfloat16_rn(v);
-}
-
 // ---------------------------------------------------------------------------
 // warp-level "reduce-scatter": on entry each lane has 32 per-head values of its
 // own row; on exit lane l holds the reduction over all 32 lanes for head l.
@@ -867,6 +860,50 @@ __device__ __forceinline__ SplitList split_list_of(const DecodeParams& p, int b,
 }
 
 }  // namespace
+
+// A finished segment's output, read by one softmax warp: its 32 heads
+// (columns from tcol) for head-dim rows `row` and 128 + `row` (O^T rows in
+// TMEM lanes), scaled per head by ev; the output (slot < 0) or the partial of a
+// split sequence (layout [slot][head][d]: a warp writes 128 contiguous bytes
+// per head). Out of line: it runs once per segment, and its code inlined in
+// the softmax loop (two or three copies) measurably slowed that loop.
+template <bool kFp8>
+__device__ __noinline__ void segment_out(float* ws_o, void* out, int out_f32, int64_t out_sb,
+                                         int64_t out_sh, int slot, int b, uint32_t tcol,
+                                         uint32_t o_lo, uint32_t o_hi, int row, int hbase,
+                                         const float* ev) {
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    const int d = half * 128 + row;
+    uint32_t r[32];
+    const uint32_t col = tcol + (half ? o_hi : o_lo);
+    tmem_ld32(col, r);
+    if (kFp8) {  // O = (V P_hi) + (V P_lo)
+      uint32_t r2[32];
+      tmem_ld32(col + 64, r2);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
+    } else {
+      tmem_wait_ld();
+    }
+    if (slot >= 0) {
+      float* dst = ws_o + static_cast<int64_t>(slot) * kPartialFloats +
+                   static_cast<int64_t>(hbase) * kDim + d;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) dst[j * kDim] = __uint_as_float(r[j]) * ev[j];
+    } else if (out_f32) {
+      float* dst = static_cast<float*>(out) + b * out_sb + hbase * out_sh + d;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) dst[j * out_sh] = __uint_as_float(r[j]) * ev[j];
+    } else {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + b * out_sb + hbase * out_sh + d;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) dst[j * out_sh] = __float2bfloat16_rn(__uint_as_float(r[j]) * ev[j]);
+    }
+  }
+}
 
 // ===========================================================================
 // the attention kernel
@@ -1378,34 +1415,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     bool have_pending = false;
     uint32_t pend_g = 0;  // tile counter of the pending segment's last tile
     auto write_segment = [&](const TileInfo& pt) {
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        const int d = half * 128 + row;
-        uint32_t r[32];
-        const uint32_t col = tmem + lane_addr + o_base<kFp8>(pt.seg, half) + hbase;
-        tmem_ld32(col, r);
-        if (kFp8) {  // O = (V P_hi) + (V P_lo)
-          uint32_t r2[32];
-          tmem_ld32(col + 64, r2);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
-        } else {
-          tmem_wait_ld();
-        }
-        if (pt.slot >= 0) {
-          // partial layout [slot][head][d]: a warp writes 128 contiguous bytes per head
-          float* dst = p.ws_o + static_cast<int64_t>(pt.slot) * kPartialFloats +
-                       static_cast<int64_t>(hbase) * kDim + d;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) dst[j * kDim] = __uint_as_float(r[j]) * ev[j];
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            store_out(p, pt.b, hbase + j, d, __uint_as_float(r[j]) * ev[j]);
-        }
-      }
+      segment_out<kFp8>(p.ws_o, p.out, p.out_f32, p.out_sb, p.out_sh, pt.slot, pt.b,
+                        tmem + lane_addr + hbase, o_base<kFp8>(pt.seg, 0), o_base<kFp8>(pt.seg, 1),
+                        row, hbase, ev);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) smem_add_release(&c.seg_arrivals, 1u);
@@ -1567,8 +1579,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // ---- output of the previous segment, deferred to here ---------------
       // Its last PV completed before this tile's P went out (the o_full wait
       // above) and the MMA now accumulates into the other O pair, so the
-      // read-out overlaps this tile's PV and the next tile's QK.
-      if (have_pending) {
+      // read-out overlaps this tile's PV and the next tile's QK. (An FP8
+      // segment is read out at its end or after the loop, never here: the
+      // condition keeps this copy of the read-out out of the FP8 loop's code.)
+      if (!kFp8 && have_pending) {
         write_segment(pend);
         have_pending = false;
       }
@@ -1642,8 +1656,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 //
 // The kernel starts while the attention kernel still runs (on SMs it has
 // left) and merges each sequence as soon as its ready word says its partials
-// are written, so merges overlap the attention kernel's last tiles. It waits
-// for the attention grid to complete only at its end, so a call is over when
+// are written, so merges overlap the attention kernel's last tiles. One CTA
+// waits for the attention grid to complete at its end, so a call is over when
 // this kernel is.
 // ===========================================================================
 __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams p) {
