@@ -257,15 +257,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (p.mode == 0 && ready) {
     // deterministic split-K merge by the last CTA to finish this output tile
-    __threadfence();
+    // (one acquire-release add per CTA, as in the fused kernel)
     __syncthreads();
     if (tid == 0) {
-      const int prev = atomicAdd(p.counters + m_tile, 1);
+      const int prev = atom_add_acq_rel_gpu(p.counters + m_tile, 1);
       c.is_last = (prev == p.splits - 1);
     }
     __syncthreads();
     if (c.is_last) {
-      __threadfence();
       merge_latent<2>(p.partials, p.splits, B, p.m_total, m, p.latent);
       if (tid == 0) p.counters[m_tile] = 0;
     }
@@ -399,10 +398,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       // the whole latent exists once every latent tile is merged (bounded);
       // every lane reads the same words, so the warp leaves the loop together
       auto await_latent = [&]() -> bool {
-        volatile int* done = p.counters + kQprojDone;
+        const int* done = p.counters + kQprojDone;
         const uint64_t t0 = global_timer_ns();
         bool good = true;
-        while (*done < p.m1_tiles) {
+        while (ld_acquire_gpu(done) < p.m1_tiles) {  // acquires the latent tiles
           if (*abort_flag) {
             good = false;
             break;
@@ -417,8 +416,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           }
         }
         if (!__all_sync(0xffffffffu, good)) return false;
-        __threadfence();             // acquire the latent tiles
-        fence_proxy_async_global();  // ... for the TMA reads that follow
+        fence_proxy_async_global();  // the acquired latent, for the TMA reads that follow
         // count this CTA as having seen the latent; the last one (after all
         // latent tiles and every other reader) returns the count to zero
         if (lane == 0 && atomicAdd(p.counters + kQprojDone, 1) == p.m1_tiles + p.m2_tiles - 1)
@@ -510,22 +508,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                 __uint_as_float(r[j]);
       }
     }
-    // deterministic split-K merge by the last CTA of this latent tile
-    __threadfence();
+    // deterministic split-K merge by the last CTA of this latent tile: one
+    // acquire-release add per CTA (its release half publishes this CTA's
+    // partial, made CTA-wide by the barrier; its acquire half the others')
     epi_sync();
     if (etid == 0) {
-      const int prev = atomicAdd(p.counters + tile1, 1);
+      const int prev = atom_add_acq_rel_gpu(p.counters + tile1, 1);
       c.is_last = (prev == p.splits - 1);
     }
     epi_sync();
     if (c.is_last) {
-      __threadfence();
       merge_latent_x4(p.partials, p.splits, B, p.rank, tile1 * 128, etid, p.latent);
-      __threadfence();
       epi_sync();
       if (etid == 0) {
         p.counters[tile1] = 0;
-        atomicAdd(p.counters + kQprojDone, 1);  // this latent tile is complete
+        red_add_release_gpu(p.counters + kQprojDone, 1);  // this latent tile is complete
       }
     }
   }

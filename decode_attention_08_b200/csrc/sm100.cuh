@@ -400,6 +400,25 @@ __device__ __forceinline__ void tma_load_4d_warp(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// GPU-scope acquire/release atomics and loads on global memory. A release by
+// one thread also publishes the writes of the threads it has synchronised
+// with before (a CTA barrier), so one thread can publish a whole CTA's stores.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // mbar_wait for a whole warp: every lane returns the same result.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
                                                volatile int* abort_flag) {
