@@ -30,6 +30,9 @@
  * bottleneck") is q = (x * W_qa) * W_qb with no bias, norm or activation, all in
  * float64 from the bf16 inputs.
  *
+ * The key/value append (below) projects the new token's hidden state into the
+ * shared K and V heads and stores the rounded rows into the cache.
+ *
  * Every input arrives as the exact bit pattern the GPU sees (bf16 bits or E4M3
  * codes) and is up-converted exactly to double here; all arithmetic is double.
  *
@@ -216,6 +219,68 @@ void mfa_oracle_query_proj(int B, int Dm, int R, int N, const uint16_t* x,
         }
     }
     free(c);
+}
+
+/*
+ * New-token key/value projection and cache append. The pages print no W_k or
+ * W_v; the plain reading of "one shared key head and one shared value head of
+ * dimension 256" fed by the 7168-wide hidden state is k = x * W_k and
+ * v = x * W_v ([B][Dm] x [Dm][D], no bias), in double from the bf16 inputs.
+ */
+void mfa_oracle_kv_project(int B, int Dm, int D, const uint16_t* x, const uint16_t* w_k,
+                           const uint16_t* w_v, double* k_out, double* v_out) {
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < D; ++i) {
+        for (int b = 0; b < B; ++b) {
+            double ak = 0.0, av = 0.0;
+            for (int k = 0; k < Dm; ++k) {
+                const double xv = bf16_bits_to_double(x[(int64_t)b * Dm + k]);
+                ak += xv * bf16_bits_to_double(w_k[(int64_t)k * D + i]);
+                av += xv * bf16_bits_to_double(w_v[(int64_t)k * D + i]);
+            }
+            k_out[(int64_t)b * D + i] = ak;
+            v_out[(int64_t)b * D + i] = av;
+        }
+    }
+}
+
+/* The bf16 nearest to v (ties to even), as bits: 8 significant bits, exponent
+ * range of binary32 (subnormals below 2^-126; beyond the largest finite value
+ * the result is infinity). */
+uint16_t mfa_oracle_bf16_round(double v) {
+    if (isnan(v)) return 0x7FC0;
+    const uint16_t sign = signbit(v) ? 0x8000 : 0;
+    const double a = fabs(v);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);     /* a = f * 2^e, f in [0.5, 1): the leading bit has weight 2^(e-1) */
+    int lead = e - 1;
+    if (lead < -126) lead = -126; /* subnormal range: fixed quantum 2^-133 */
+    double r = nearbyint(ldexp(a, 7 - lead)); /* significand in units of the last bit, ties to even */
+    double q = ldexp(r, lead - 7);            /* the rounded magnitude */
+    if (q >= ldexp(1.0, 128)) return sign | 0x7F80;
+    float f = (float)q; /* exact: q has at most 8 significant bits in binary32's range */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
+}
+
+/* The E4M3 code nearest to v (ties to the code with an even mantissa),
+ * saturating to +-448 beyond it; NaN to 0x7F. Searches all finite codes. */
+uint8_t mfa_oracle_e4m3_encode(double v) {
+    if (isnan(v)) return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0;
+    const double a = fabs(v);
+    int best = 0;
+    double best_d = INFINITY;
+    for (int code = 0; code <= 0x7E; ++code) {
+        const double d = fabs(mfa_oracle_e4m3_to_double((uint8_t)code) - a);
+        if (d < best_d || (d == best_d && (code & 1) == 0)) {
+            best_d = d;
+            best = code;
+        }
+    }
+    return (uint8_t)(sign | best);
 }
 
 /* Number of OpenMP threads a parallel region here would use (1 without OpenMP). */

@@ -90,3 +90,8 @@ def combine(parts, part_lse):
 def query_proj(x_bits, wqa_bits, wqb_bits):
     x = bf16_bits_to_f64(x_bits)
     return (x @ bf16_bits_to_f64(wqa_bits)) @ bf16_bits_to_f64(wqb_bits)
+
+
+def kv_project(x_bits, wk_bits, wv_bits):
+    x = bf16_bits_to_f64(x_bits)
+    return x @ bf16_bits_to_f64(wk_bits), x @ bf16_bits_to_f64(wv_bits)

@@ -54,6 +54,12 @@ def _load():
             lib.mfa_oracle_query_proj.argtypes = [ctypes.c_int] * 4 + [P, P, P, P]
             lib.mfa_oracle_e4m3_to_double.restype = ctypes.c_double
             lib.mfa_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            lib.mfa_oracle_kv_project.restype = None
+            lib.mfa_oracle_kv_project.argtypes = [ctypes.c_int] * 3 + [P, P, P, P, P]
+            lib.mfa_oracle_bf16_round.restype = ctypes.c_uint16
+            lib.mfa_oracle_bf16_round.argtypes = [ctypes.c_double]
+            lib.mfa_oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.mfa_oracle_e4m3_encode.argtypes = [ctypes.c_double]
             lib.mfa_oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -149,3 +155,60 @@ def query_proj(x_bits, wqa_bits, wqb_bits):
     out = np.zeros((B, N), np.float64)
     lib.mfa_oracle_query_proj(B, Dm, R, N, _ptr(x_bits), _ptr(wqa_bits), _ptr(wqb_bits), _ptr(out))
     return out
+
+
+def bf16_round(v: float) -> int:
+    """Bits of the bf16 nearest to v (ties to even)."""
+    return int(_load().mfa_oracle_bf16_round(float(v)))
+
+
+def e4m3_encode(v: float) -> int:
+    """The E4M3 code nearest to v (ties to an even mantissa, saturating to +-448)."""
+    return int(_load().mfa_oracle_e4m3_encode(float(v)))
+
+
+def kv_project(x_bits, wk_bits, wv_bits):
+    """k = x @ W_k, v = x @ W_v in float64 from bf16 bits; x [B, Dm], W [Dm, D]."""
+    lib = _load()
+    x_bits = _c(x_bits, np.uint16)
+    wk_bits = _c(wk_bits, np.uint16)
+    wv_bits = _c(wv_bits, np.uint16)
+    B, Dm = x_bits.shape
+    assert wk_bits.shape == wv_bits.shape and wk_bits.shape[0] == Dm
+    D = wk_bits.shape[1]
+    k = np.zeros((B, D), np.float64)
+    v = np.zeros((B, D), np.float64)
+    lib.mfa_oracle_kv_project(B, Dm, D, _ptr(x_bits), _ptr(wk_bits), _ptr(wv_bits), _ptr(k), _ptr(v))
+    return k, v
+
+
+def kv_append(x_bits, wk_bits, wv_bits, k_cache, v_cache, positions, *, kv_dtype=BF16,
+              page_table=None, page_size=64, k_scale=1.0, v_scale=1.0):
+    """The caches after appending each sequence's new token at row positions[b].
+
+    k_cache, v_cache: contiguous [B, Lmax, D] or paged [num_pages, page_size, D],
+    uint16 (bf16 bits) or uint8 (E4M3 codes); page_table int32 [B, max_pages].
+    A bf16 cache stores the nearest bf16 of the projected value, an FP8 cache the
+    E4M3 code nearest to value / scale. Returns (k_new, v_new, k, v): updated
+    copies of the caches and the projected rows in float64.
+    """
+    k, v = kv_project(x_bits, wk_bits, wv_bits)
+    k_new = np.array(k_cache, copy=True)
+    v_new = np.array(v_cache, copy=True)
+    B, D = k.shape
+    for b in range(B):
+        t = int(positions[b])
+        if page_table is not None:
+            page = int(page_table[b][t // page_size])
+            if page < 0 or page >= k_new.shape[0]:
+                raise ValueError("oracle: out-of-range page id")
+            rows = (k_new[page, t % page_size], v_new[page, t % page_size])
+        else:
+            if t < 0 or t >= k_new.shape[1]:
+                raise ValueError("oracle: position outside the cache")
+            rows = (k_new[b, t], v_new[b, t])
+        for dst, val, scale in ((rows[0], k[b], k_scale), (rows[1], v[b], v_scale)):
+            for i in range(D):
+                dst[i] = (e4m3_encode(val[i] / scale) if kv_dtype == E4M3
+                          else bf16_round(val[i]))
+    return k_new, v_new, k, v
