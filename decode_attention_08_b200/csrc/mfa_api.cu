@@ -21,6 +21,8 @@ cudaError_t launch_qproj_fused(const CUtensorMap& twa, const CUtensorMap& tx,
                                const QprojFusedParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_qproj(const CUtensorMap& tw, const CUtensorMap& ta, const QprojParams& p,
                          int m_tiles, cudaStream_t stream);
+cudaError_t launch_kv_append(const CUtensorMap& twk, const CUtensorMap& twv, const CUtensorMap& tx,
+                             const QprojParams& pg, const KvAppendParams& pm, cudaStream_t stream);
 }  // namespace mfa
 
 using namespace mfa;
@@ -719,3 +721,137 @@ extern "C" int mfa_decode_attention_noalloc(const mfa_tensor* q, const mfa_tenso
                      k_scale, v_scale, num_splits, lse_out, scratch, kNoAllocScratchBytes, stream,
                      false);
 }
+
+// ===========================================================================
+// New-token key/value projection and cache append
+// ===========================================================================
+namespace {
+
+// Split-K factor of the append projection: the four 128-feature tiles of
+// [W_k | W_v] times this many k-ranges fill the SMs.
+int kv_append_splits(int64_t hidden, int sms) {
+  int s = sms / 4;
+  if (s < 1) s = 1;
+  if (s > hidden / 64) s = static_cast<int>(hidden / 64);
+  return s;
+}
+
+size_t kv_append_ws_bytes(int64_t batch, int64_t hidden, int sms) {
+  return align256(static_cast<size_t>(kv_append_splits(hidden, sms)) * batch * 2 * kDim *
+                  sizeof(float));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mfa_kv_append_workspace_size(int batch, int hidden) {
+  if (batch <= 0 || hidden <= 0 || hidden % 64) return 0;
+  DeviceInfo d;
+  const int rc = current_device(&d);
+  if (rc != MFA_OK && rc != MFA_ERR_UNSUPPORTED) return 0;
+  return kv_append_ws_bytes(batch, hidden, d.sms);
+}
+
+int mfa_kv_append(const mfa_tensor* x, const mfa_tensor* w_k, const mfa_tensor* w_v,
+                  mfa_tensor* k_cache, mfa_tensor* v_cache, const mfa_tensor* page_table,
+                  const mfa_tensor* positions, int kv_dtype, float k_scale, float v_scale,
+                  void* workspace, size_t workspace_bytes, mfa_stream_t stream) {
+  // ---- shapes and dtypes ----
+  if (!well_formed(x, 2) || !well_formed(w_k, 2) || !well_formed(w_v, 2) ||
+      !well_formed(k_cache, 3) || !well_formed(v_cache, 3) || !well_formed(positions, 1))
+    return MFA_ERR_INVALID_ARG;
+  for (const mfa_tensor* t : std::initializer_list<const mfa_tensor*>{x, w_k, w_v})
+    if (t->dtype != MFA_BF16 || t->stride[1] != 1 || t->stride[0] % 8 || !aligned16(t->data))
+      return MFA_ERR_INVALID_ARG;
+  const int64_t B = x->shape[0], Dm = x->shape[1];
+  if (w_k->shape[0] != Dm || w_v->shape[0] != Dm || w_k->shape[1] != kDim ||
+      w_v->shape[1] != kDim)
+    return MFA_ERR_INVALID_ARG;
+  if (B < 1 || B > 256 || Dm <= 0 || Dm % 64 || Dm > (1 << 20)) return MFA_ERR_UNSUPPORTED;
+  if (kv_dtype != MFA_BF16 && kv_dtype != MFA_FP8_E4M3) return MFA_ERR_INVALID_ARG;
+  if (k_cache->dtype != kv_dtype || v_cache->dtype != kv_dtype) return MFA_ERR_INVALID_ARG;
+  if (!(k_scale == k_scale) || !(v_scale == v_scale)) return MFA_ERR_INVALID_ARG;
+  if (kv_dtype == MFA_BF16 && (k_scale != 1.f || v_scale != 1.f)) return MFA_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || k_scale > 1e30f || v_scale > 1e30f)
+    return MFA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (k_cache->shape[i] != v_cache->shape[i] || k_cache->stride[i] != v_cache->stride[i])
+      return MFA_ERR_INVALID_ARG;
+  if (k_cache->shape[2] != kDim || k_cache->stride[2] != 1) return MFA_ERR_INVALID_ARG;
+  if (!k_cache->data || !v_cache->data) return MFA_ERR_INVALID_ARG;
+  if (positions->dtype != MFA_I32 || positions->shape[0] != B || positions->stride[0] != 1)
+    return MFA_ERR_INVALID_ARG;
+  const bool paged = page_table != nullptr;
+  int page_size = 0, max_pages = 0, num_pages = 0;
+  int64_t cap = 0;
+  if (paged) {
+    if (!well_formed(page_table, 2) || page_table->dtype != MFA_I32 ||
+        page_table->shape[0] != B || page_table->stride[1] != 1)
+      return MFA_ERR_INVALID_ARG;
+    if (k_cache->shape[0] <= 0 || k_cache->shape[0] > (1ll << 31) - 1 || k_cache->shape[1] <= 0 ||
+        k_cache->shape[1] > (1 << 20) || page_table->shape[1] <= 0 ||
+        page_table->shape[1] > (1 << 24))
+      return MFA_ERR_INVALID_ARG;
+    page_size = static_cast<int>(k_cache->shape[1]);
+    num_pages = static_cast<int>(k_cache->shape[0]);
+    max_pages = static_cast<int>(page_table->shape[1]);
+    if (static_cast<int64_t>(max_pages) * page_size > (1ll << 30)) return MFA_ERR_UNSUPPORTED;
+  } else {
+    if (k_cache->shape[0] != B) return MFA_ERR_INVALID_ARG;
+    cap = k_cache->shape[1];
+    if (cap > (1 << 30)) return MFA_ERR_UNSUPPORTED;
+  }
+
+  DeviceInfo dev;
+  int rc = current_device(&dev);
+  if (rc != MFA_OK) return rc;
+  const int splits = kv_append_splits(Dm, dev.sms);
+  if (!workspace || workspace_bytes < kv_append_ws_bytes(B, Dm, dev.sms) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return MFA_ERR_WORKSPACE;
+
+  const int n_cols = static_cast<int>((B + 15) / 16 * 16);
+  CUtensorMap twk, twv, tx;
+  if (encode_2d(&twk, w_k->data, kDim, Dm, w_k->stride[0], 64, 64) != CUDA_SUCCESS ||
+      encode_2d(&twv, w_v->data, kDim, Dm, w_v->stride[0], 64, 64) != CUDA_SUCCESS ||
+      encode_2d(&tx, x->data, Dm, B, x->stride[0], 64, n_cols) != CUDA_SUCCESS)
+    return MFA_ERR_INVALID_ARG;
+
+  QprojParams pg;
+  std::memset(&pg, 0, sizeof pg);
+  pg.batch = static_cast<int>(B);
+  pg.k_blocks = static_cast<int>(Dm / 64);
+  pg.m_total = 2 * kDim;
+  pg.splits = splits;
+  pg.n_cols = n_cols;
+  pg.mode = 2;
+  pg.partials = static_cast<float*>(workspace);
+  pg.m_half = kDim / 128;
+
+  KvAppendParams pm;
+  std::memset(&pm, 0, sizeof pm);
+  pm.batch = static_cast<int>(B);
+  pm.splits = splits;
+  pm.partials = static_cast<const float*>(workspace);
+  pm.k_cache = k_cache->data;
+  pm.v_cache = v_cache->data;
+  pm.fp8 = kv_dtype == MFA_FP8_E4M3;
+  pm.k_scale = k_scale;
+  pm.v_scale = v_scale;
+  pm.positions = static_cast<const int*>(positions->data);
+  pm.page_table = paged ? static_cast<const int*>(page_table->data) : nullptr;
+  pm.pt_stride = paged ? page_table->stride[0] : 0;
+  pm.page_size = page_size;
+  pm.max_pages = max_pages;
+  pm.num_pages = num_pages;
+  pm.cache_bs = k_cache->stride[0];
+  pm.cache_ts = k_cache->stride[1];
+  pm.cap_tokens = static_cast<int>(cap);
+
+  const cudaError_t e =
+      launch_kv_append(twk, twv, tx, pg, pm, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MFA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

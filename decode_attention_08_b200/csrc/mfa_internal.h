@@ -76,6 +76,27 @@ struct QprojParams {
   __nv_bfloat16* latent; // [2 * batch][m_total], rows 2j / 2j+1 = high part / residual
   __nv_bfloat16* q_out;  // (mode 1 output)
   int64_t q_stride;      // elements between q_out rows
+  // mode 2 (key/value append): output tiles m < m_half come from the first
+  // weight map (W_k), the others from the second (W_v); partials only
+  int m_half;
+};
+
+// Key/value append: the rows of the new tokens, merged from the split-K
+// partials of the projection and stored into the caches.
+struct KvAppendParams {
+  int batch;
+  int splits;
+  const float* partials;   // [splits][batch][2 * kDim] (k features, then v features)
+  void* k_cache;
+  void* v_cache;
+  int fp8;                 // caches hold E4M3 codes (else bf16)
+  float k_scale, v_scale;  // FP8: stored code = E4M3(value / scale)
+  const int* positions;    // [batch] row of each sequence's new token
+  const int* page_table;   // [batch][max_pages], or null for contiguous caches
+  int64_t pt_stride;
+  int page_size, max_pages, num_pages;
+  int64_t cache_bs, cache_ts;  // element strides of a sequence (page, if paged) and a token row
+  int cap_tokens;              // contiguous caches: rows per sequence
 };
 
 // Both projection GEMMs in one persistent kernel (small batches): split-K

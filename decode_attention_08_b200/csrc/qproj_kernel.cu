@@ -140,7 +140,8 @@ __device__ __forceinline__ void merge_latent_x4(const float* partials, int split
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mfa_qproj_kernel(const __grid_constant__ CUtensorMap tm_w,
-                     const __grid_constant__ CUtensorMap tm_act, const QprojParams p) {
+                     const __grid_constant__ CUtensorMap tm_act,
+                     const __grid_constant__ CUtensorMap tm_w2, const QprojParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -180,7 +181,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------- producer ----------------
     const uint64_t pol_w = l2_policy_evict_first();
     const uint64_t pol_a = l2_policy_evict_last();
-    tma_prefetch_desc(&tm_w);
+    // mode 2: tiles from m_half on are the second weight's (W_v)
+    const bool second = p.mode == 2 && m_tile >= p.m_half;
+    const CUtensorMap* wm = second ? &tm_w2 : &tm_w;
+    const int wcol = (second ? m_tile - p.m_half : m_tile) * 128;
+    tma_prefetch_desc(wm);
     tma_prefetch_desc(&tm_act);
     for (int i = 0; i < nkb; ++i) {
       const int s = i % stages;
@@ -188,8 +193,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint8_t* st = smem + s * stage_bytes;
       mbar_arrive_expect_tx(&c.full[s], stage_bytes);
       const int kb = kb0 + i;
-      tma_load_2d(st, &tm_w, &c.full[s], m_tile * 128, kb * 64, pol_w);
-      tma_load_2d(st + kABytes / 2, &tm_w, &c.full[s], m_tile * 128 + 64, kb * 64, pol_w);
+      tma_load_2d(st, wm, &c.full[s], wcol, kb * 64, pol_w);
+      tma_load_2d(st + kABytes / 2, wm, &c.full[s], wcol + 64, kb * 64, pol_w);
       tma_load_2d(st + kABytes, &tm_act, &c.full[s], kb * 64, 0, pol_a);
     }
   } else if (warp == 1) {
@@ -223,7 +228,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const int B = p.batch;
   if (ready) {
-    if (p.mode == 0) {
+    if (p.mode == 0 || p.mode == 2) {
       for (int cb = 0; cb < n_cols; cb += 16) {
         uint32_t r[16];
         tmem_ld16(taddr + cb, r);
@@ -583,9 +588,96 @@ cudaError_t launch_qproj(const CUtensorMap& tw, const CUtensorMap& ta, const Qpr
   cudaError_t err =
       cudaFuncSetAttribute(mfa_qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  dim3 grid(m_tiles, p.mode == 0 ? p.splits : 1);
-  mfa_qproj_kernel<<<grid, kGemmThreads, smem, stream>>>(tw, ta, p);
+  dim3 grid(m_tiles, p.mode == 1 ? 1 : p.splits);
+  mfa_qproj_kernel<<<grid, kGemmThreads, smem, stream>>>(tw, ta, tw, p);
   return cudaGetLastError();
+}
+
+// ===========================================================================
+// Key/value append: the projection x [W_k | W_v] as split-K partials (the GEMM
+// above in mode 2, tiles of W_k then W_v), then a merge kernel in which a
+// thread owns one (sequence, feature) output: it sums the splits in order (as
+// deterministic as the latent merge) and stores the value into the cache row
+// of the sequence's new token -- the nearest bf16, or the E4M3 code nearest to
+// value / scale (saturating) for an FP8 cache -- through the page table when
+// there is one. Positions and page ids are checked; a bad one is recorded as
+// MFA_ERR_BAD_INDEX and its row is not written.
+// ===========================================================================
+constexpr int kMergeThreads = 256;
+constexpr int kAppendSplitBatch = 8;  // partial loads in flight per thread
+
+__global__ void __launch_bounds__(kMergeThreads)
+    mfa_kv_merge_kernel(const KvAppendParams p) {
+  griddep_wait();  // the partials of the projection kernel
+  constexpr int kFeat = 2 * kDim;
+  const int64_t o = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
+  if (o >= static_cast<int64_t>(p.batch) * kFeat) return;
+  const int b = static_cast<int>(o / kFeat);
+  const int f = static_cast<int>(o % kFeat);
+  float acc = 0.f;
+  for (int s0 = 0; s0 < p.splits; s0 += kAppendSplitBatch) {
+    float v[kAppendSplitBatch];
+#pragma unroll
+    for (int u = 0; u < kAppendSplitBatch; ++u)
+      v[u] = s0 + u < p.splits
+                 ? __ldcg(p.partials + (static_cast<int64_t>(s0 + u) * p.batch + b) * kFeat + f)
+                 : 0.f;
+#pragma unroll
+    for (int u = 0; u < kAppendSplitBatch; ++u)
+      if (s0 + u < p.splits) acc += v[u];
+  }
+  const bool is_v = f >= kDim;
+  const int d = is_v ? f - kDim : f;
+  const int t = p.positions[b];
+  int64_t row;  // element offset of the new token's row
+  if (p.page_table) {
+    if (t < 0 || t >= p.max_pages * p.page_size) {
+      record_error(5 /* MFA_ERR_BAD_INDEX */);
+      return;
+    }
+    const int page = p.page_table[static_cast<int64_t>(b) * p.pt_stride + t / p.page_size];
+    if (page < 0 || page >= p.num_pages) {
+      record_error(5 /* MFA_ERR_BAD_INDEX */);
+      return;
+    }
+    row = static_cast<int64_t>(page) * p.cache_bs + static_cast<int64_t>(t % p.page_size) * p.cache_ts;
+  } else {
+    if (t < 0 || t >= p.cap_tokens) {
+      record_error(5 /* MFA_ERR_BAD_INDEX */);
+      return;
+    }
+    row = static_cast<int64_t>(b) * p.cache_bs + static_cast<int64_t>(t) * p.cache_ts;
+  }
+  void* cache = is_v ? p.v_cache : p.k_cache;
+  if (p.fp8) {
+    const float scaled = acc / (is_v ? p.v_scale : p.k_scale);
+    static_cast<uint8_t*>(cache)[row + d] =
+        static_cast<uint8_t>(__nv_cvt_float_to_fp8(scaled, __NV_SATFINITE, __NV_E4M3));
+  } else {
+    static_cast<__nv_bfloat16*>(cache)[row + d] = __float2bfloat16_rn(acc);
+  }
+}
+
+cudaError_t launch_kv_append(const CUtensorMap& twk, const CUtensorMap& twv, const CUtensorMap& tx,
+                             const QprojParams& pg, const KvAppendParams& pm, cudaStream_t stream) {
+  const int smem = qproj_smem_bytes(pg.n_cols);
+  cudaError_t err =
+      cudaFuncSetAttribute(mfa_qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  mfa_qproj_kernel<<<dim3(2 * pg.m_half, pg.splits), kGemmThreads, smem, stream>>>(twk, tx, twv, pg);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t outputs = static_cast<int64_t>(pm.batch) * 2 * kDim;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((outputs + kMergeThreads - 1) / kMergeThreads));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mfa_kv_merge_kernel, pm);
 }
 
 }  // namespace mfa

@@ -161,6 +161,22 @@ def make_proj_inputs(seed: int, batch: int, hidden: int = HIDDEN, rank: int = RA
     return ProjInputs(x=x, w_qa=w_qa, w_qb=w_qb)
 
 
+@dataclass
+class KvAppendInputs:
+    x: torch.Tensor    # [B, hidden] bf16 hidden states of the new tokens
+    w_k: torch.Tensor  # [hidden, 256] bf16
+    w_v: torch.Tensor  # [hidden, 256] bf16
+
+
+def make_kv_append_inputs(seed: int, batch: int, hidden: int = HIDDEN) -> KvAppendInputs:
+    """Hidden states ~ N(0, 1) and key/value weights ~ N(0, 0.02), as the projection's."""
+    g = torch.Generator().manual_seed(int(seed))
+    x = _randn_bf16(g, (batch, hidden))
+    w_k = _randn_bf16(g, (hidden, D), std=0.02)
+    w_v = _randn_bf16(g, (hidden, D), std=0.02)
+    return KvAppendInputs(x=x, w_k=w_k, w_v=w_v)
+
+
 # The five workloads (seed = 1000 + index). Index 2 is the headline workload.
 WORKLOADS = {
     1: dict(name="mfa_decode_b1_l512_bf16", batch=1, seq_len=512),

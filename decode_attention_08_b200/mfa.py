@@ -42,6 +42,7 @@ _lock = threading.Lock()
 
 EXPORTS = ("mfa_decode_attention", "mfa_decode_attention_ex", "mfa_decode_workspace_size",
            "mfa_query_proj", "mfa_query_proj_ex", "mfa_query_proj_workspace_size",
+           "mfa_kv_append", "mfa_kv_append_workspace_size",
            "mfa_read_status", "mfa_error_string", "mfa_version", "mfa_last_cuda_error_string",
            "mfa_decode_attention_noalloc")
 
@@ -75,6 +76,11 @@ def lib() -> ctypes.CDLL:
             L.mfa_query_proj_ex.restype = ctypes.c_int
             L.mfa_query_proj_workspace_size.argtypes = [ctypes.c_int] * 3
             L.mfa_query_proj_workspace_size.restype = ctypes.c_size_t
+            L.mfa_kv_append.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_float,
+                                        ctypes.c_float, P, ctypes.c_size_t, P]
+            L.mfa_kv_append.restype = ctypes.c_int
+            L.mfa_kv_append_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int]
+            L.mfa_kv_append_workspace_size.restype = ctypes.c_size_t
             L.mfa_read_status.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
             L.mfa_read_status.restype = ctypes.c_int
             L.mfa_error_string.argtypes = [ctypes.c_int]
@@ -193,6 +199,30 @@ def query_proj_ex(x, w_qa, w_qb, q_out, workspace: torch.Tensor, stream=None):
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "mfa_query_proj_ex")
     return q_out
+
+
+def kv_append_workspace_size(batch: int, hidden: int) -> int:
+    return int(lib().mfa_kv_append_workspace_size(int(batch), int(hidden)))
+
+
+def kv_append(x, w_k, w_v, k_cache, v_cache, positions, page_table=None, kv_dtype="bf16",
+              k_scale: float = 1.0, v_scale: float = 1.0, workspace=None, stream=None):
+    """``mfa_kv_append``: writes each sequence's new key/value row (x W_k, x W_v)
+    into the caches at row ``positions[b]``. ``workspace`` is allocated here when
+    not given."""
+    if workspace is None:
+        n = kv_append_workspace_size(x.shape[0], x.shape[1])
+        if n == 0:
+            raise RuntimeError("mfa_kv_append_workspace_size failed")
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device)
+    rc = lib().mfa_kv_append(describe(x), describe(w_k), describe(w_v), describe(k_cache),
+                             describe(v_cache),
+                             None if page_table is None else describe(page_table),
+                             describe(positions), _kv_code(kv_dtype), float(k_scale),
+                             float(v_scale), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mfa_kv_append")
+    return k_cache, v_cache
 
 
 def read_status(stream=None, reset: bool = True) -> int:

@@ -192,6 +192,42 @@ int mfa_query_proj_ex(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_ten
 
 size_t mfa_query_proj_workspace_size(int batch, int dm, int rank);
 
+/*
+ * New-token key/value projection and cache append. The Step-3 page (Key points
+ * -> Architecture) gives every token one shared key head and one shared value
+ * head of dimension 256 fed by the 7168-wide hidden state; it prints no W_k or
+ * W_v, and the plain reading is k = x * W_k, v = x * W_v (no bias, norm or
+ * positional transform). Each sequence b's new row is written at token index
+ * positions[b] of its cache -- the row the next decode-attention call reads
+ * once seq_lens[b] = positions[b] + 1.
+ *
+ *  x          [B, Dm] bf16 hidden states of the new tokens (row stride a multiple of 8).
+ *  w_k, w_v   [Dm, 256] bf16 row-major.
+ *  k_cache, v_cache  the caches of mfa_decode_attention (contiguous [B, Lmax, 256]
+ *             or paged [num_pages, page_size, 256]), same shape and strides,
+ *             dtype kv_dtype; a bf16 cache takes the nearest bf16 of the
+ *             projected value, an E4M3 cache the E4M3 code nearest to
+ *             value / k_scale (resp. v_scale), saturating to +-448.
+ *  page_table [B, max_pages] int32 (device) or NULL for contiguous caches.
+ *  positions  [B] int32 (device): the row of each sequence's new token.
+ *  k_scale, v_scale  > 0; must be 1 for bf16 caches.
+ *  workspace  at least mfa_kv_append_workspace_size(B, Dm) bytes, 256-byte
+ *             aligned, no initialisation needed (it holds split-K partials).
+ * 1 <= B <= 256; Dm a multiple of 64. The projection accumulates in fp32 (split
+ * over the hidden dimension, partials summed in a fixed order, so results do
+ * not depend on timing) and rounds once, on store. Two kernels on `stream`.
+ * A position outside the cache or a page id outside [0, num_pages) is not
+ * written and is reported later by mfa_read_status as MFA_ERR_BAD_INDEX.
+ * Returns MFA_OK, MFA_ERR_INVALID_ARG, MFA_ERR_UNSUPPORTED, MFA_ERR_WORKSPACE
+ * or MFA_ERR_CUDA (then nothing was launched, or a launch failed).
+ */
+int mfa_kv_append(const mfa_tensor* x, const mfa_tensor* w_k, const mfa_tensor* w_v,
+                  mfa_tensor* k_cache, mfa_tensor* v_cache, const mfa_tensor* page_table,
+                  const mfa_tensor* positions, int kv_dtype, float k_scale, float v_scale,
+                  void* workspace, size_t workspace_bytes, mfa_stream_t stream);
+
+size_t mfa_kv_append_workspace_size(int batch, int hidden);
+
 /* Synchronises `stream`, then reads (and, if reset != 0, clears) the current
  * device's status word: MFA_OK or the first MFA_ERR_BAD_INDEX / MFA_ERR_TIMEOUT
  * a kernel recorded since the last reset. Returns MFA_OK or MFA_ERR_CUDA. */
