@@ -410,6 +410,9 @@ def other_workloads(hbm_peak: float):
         res[gen.WORKLOADS[idx]["name"]] = entry
         del step
         torch.cuda.empty_cache()
+    for batch, kv in ((64, "bf16"), (128, "e4m3")):
+        res[f"mfa_kv_append_b{batch}_h7168_{kv}"] = time_kv_append(batch, kv, hbm_peak)
+        torch.cuda.empty_cache()
     return res
 
 
@@ -449,6 +452,61 @@ def time_qproj(proj: gen.ProjInputs, hbm_peak: float):
     return {"us_per_call": t * 1e6, "alg_bytes": alg, "gbs": alg / t / 1e9,
             "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak, "tflops": flops / t / 1e12,
             "note": "batch <= 8: one persistent kernel (split-K latent GEMM, deterministic merge, up-projection whose weights fill the ring while the latent forms); larger batches: two launches"}
+
+
+def time_kv_append(batch: int, kv_dtype: str, hbm_peak: float):
+    """The new token's key/value projection and cache append of a decode batch
+    (contiguous cache of 4097 rows per sequence, row 4096 written). The weights
+    rotate through 20 device copies (147 MB > L2): in a decode step the other
+    layers' weights pass through L2 between two appends of one layer."""
+    from decode_attention_08_b200 import mfa
+    inp = gen.make_kv_append_inputs(3000 + batch, batch)
+    x = inp.x.cuda()
+    copies = [(inp.w_k.cuda(), inp.w_v.cuda()) for _ in range(20)]
+    fp8 = kv_dtype == "e4m3"
+    shape = (batch, 4097, 256)
+    kc = torch.zeros(shape, dtype=torch.uint8 if fp8 else torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    pos = torch.full((batch,), 4096, dtype=torch.int32, device="cuda")
+    ws = torch.empty(mfa.kv_append_workspace_size(batch, x.shape[1]), dtype=torch.uint8,
+                     device="cuda")
+    sc = (0.02, 0.02) if fp8 else (1.0, 1.0)
+    st = torch.cuda.Stream()
+
+    def call(i):
+        wk, wv = copies[i % len(copies)]
+        mfa.kv_append(x, wk, wv, kc, vc, pos, kv_dtype=kv_dtype, k_scale=sc[0], v_scale=sc[1],
+                      workspace=ws, stream=st)
+
+    with torch.cuda.stream(st):
+        for i in range(3):
+            call(i)
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(len(copies)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            call(i)
+        graphs.append(g)
+    for i in range(len(copies)):
+        graphs[i].replay()
+    torch.cuda.synchronize()
+    n = 200
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(st):
+        s.record(st)
+        for i in range(n):
+            graphs[i % len(graphs)].replay()
+        e.record(st)
+    torch.cuda.synchronize()
+    status = mfa.read_status()
+    t = s.elapsed_time(e) / 1e3 / n
+    esz = 1 if fp8 else 2
+    alg = (2 * x.shape[1] * 256 * 2 + x.numel() * 2 + batch * 2 * 256 * esz + batch * 4)
+    return {"us_per_call": t * 1e6, "alg_bytes": alg, "gbs": alg / t / 1e9,
+            "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak, "status": status,
+            "note": "split-K projection x [W_k | W_v] (one launch) + merge-and-store kernel; "
+                    "weights rotate through 20 copies (> L2)"}
 
 
 def run_ours(args, world, rank, local):
