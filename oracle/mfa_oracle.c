@@ -283,6 +283,27 @@ uint8_t mfa_oracle_e4m3_encode(double v) {
     return (uint8_t)(sign | best);
 }
 
+/*
+ * Output projection: the attention outputs of a token, its 64 heads x 256
+ * concatenated (16384 values), times W_o back to the 7168-wide hidden state:
+ * y = o * W_o ([B][K] x [K][N], no bias), in double from the bf16 inputs. The
+ * pages name no W_o; this is the plain reading of an attention layer's output
+ * projection to the hidden size.
+ */
+void mfa_oracle_out_proj(int B, int K, int N, const uint16_t* o, const uint16_t* w_o,
+                         double* y_out) {
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        for (int b = 0; b < B; ++b) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k)
+                acc += bf16_bits_to_double(o[(int64_t)b * K + k]) *
+                       bf16_bits_to_double(w_o[(int64_t)k * N + n]);
+            y_out[(int64_t)b * N + n] = acc;
+        }
+    }
+}
+
 /* Number of OpenMP threads a parallel region here would use (1 without OpenMP). */
 int mfa_oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -95,3 +95,7 @@ def query_proj(x_bits, wqa_bits, wqb_bits):
 def kv_project(x_bits, wk_bits, wv_bits):
     x = bf16_bits_to_f64(x_bits)
     return x @ bf16_bits_to_f64(wk_bits), x @ bf16_bits_to_f64(wv_bits)
+
+
+def out_proj(o_bits, wo_bits):
+    return bf16_bits_to_f64(o_bits) @ bf16_bits_to_f64(wo_bits)

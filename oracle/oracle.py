@@ -60,6 +60,8 @@ def _load():
             lib.mfa_oracle_bf16_round.argtypes = [ctypes.c_double]
             lib.mfa_oracle_e4m3_encode.restype = ctypes.c_uint8
             lib.mfa_oracle_e4m3_encode.argtypes = [ctypes.c_double]
+            lib.mfa_oracle_out_proj.restype = None
+            lib.mfa_oracle_out_proj.argtypes = [ctypes.c_int] * 3 + [P, P, P]
             lib.mfa_oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -212,3 +214,16 @@ def kv_append(x_bits, wk_bits, wv_bits, k_cache, v_cache, positions, *, kv_dtype
                 dst[i] = (e4m3_encode(val[i] / scale) if kv_dtype == E4M3
                           else bf16_round(val[i]))
     return k_new, v_new, k, v
+
+
+def out_proj(o_bits, wo_bits):
+    """y = o @ W_o in float64 from bf16 bits; o [B, K] (heads x dim), W_o [K, N]."""
+    lib = _load()
+    o_bits = _c(o_bits, np.uint16)
+    wo_bits = _c(wo_bits, np.uint16)
+    B, K = o_bits.shape
+    assert wo_bits.shape[0] == K
+    N = wo_bits.shape[1]
+    y = np.zeros((B, N), np.float64)
+    lib.mfa_oracle_out_proj(B, K, N, _ptr(o_bits), _ptr(wo_bits), _ptr(y))
+    return y

@@ -1,4 +1,5 @@
-"""Pins for the oracle's new-token key/value projection and cache append.
+"""Pins for the oracle's new-token key/value projection and cache append, and for its
+output projection.
 
 The rounding functions are pinned by hand-computed ties and landmarks of the
 formats (bf16: binary32's top half; E4M3: the OCP FP8 definition, largest
@@ -124,3 +125,26 @@ def test_kv_append_placement(oracle_mod, kv_dtype):
             assert np.array_equal(vp_new[table[b, t // ps], t % ps], v_new[b, t])
     with pytest.raises(ValueError):
         oracle_mod.kv_append(x, wk, wv, kc, vc, np.array([0, 5, L], np.int32), **kw)
+
+
+def test_output_projection_one_hot_twin_and_decimal(oracle_mod):
+    """The output projection oracle: one-hot rows select weight rows exactly, it
+    agrees with the NumPy twin, and a 50-digit evaluation on a tiny case."""
+    import decimal
+    g = torch.Generator().manual_seed(12)
+    o = torch.randn(3, 128, generator=g).to(torch.bfloat16)
+    w = torch.randn(128, 48, generator=g).to(torch.bfloat16)
+    y = oracle_mod.out_proj(gen.bits(o), gen.bits(w))
+    np.testing.assert_allclose(y, onp.out_proj(gen.bits(o), gen.bits(w)), rtol=1e-12, atol=1e-13)
+    onehot = torch.zeros(2, 128, dtype=torch.bfloat16)
+    onehot[0, 3] = 1.0
+    onehot[1, 127] = -4.0
+    y1 = oracle_mod.out_proj(gen.bits(onehot), gen.bits(w))
+    wf = w.double().numpy()
+    assert np.array_equal(y1[0], wf[3]) and np.array_equal(y1[1], -4.0 * wf[127])
+    decimal.getcontext().prec = 50
+    of, wf2 = o.double().numpy(), w.double().numpy()
+    for b, n in ((0, 0), (2, 47), (1, 20)):
+        exact = sum(decimal.Decimal(float(of[b, k])) * decimal.Decimal(float(wf2[k, n]))
+                    for k in range(128))
+        assert abs(float(exact) - y[b, n]) <= 1e-12 * max(1.0, abs(float(exact)))
