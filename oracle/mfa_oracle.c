@@ -292,14 +292,15 @@ uint8_t mfa_oracle_e4m3_encode(double v) {
  */
 void mfa_oracle_out_proj(int B, int K, int N, const uint16_t* o, const uint16_t* w_o,
                          double* y_out) {
+    /* every y[b][n] sums its K products in ascending k; W_o is walked row by row */
 #pragma omp parallel for schedule(static)
-    for (int n = 0; n < N; ++n) {
-        for (int b = 0; b < B; ++b) {
-            double acc = 0.0;
-            for (int k = 0; k < K; ++k)
-                acc += bf16_bits_to_double(o[(int64_t)b * K + k]) *
-                       bf16_bits_to_double(w_o[(int64_t)k * N + n]);
-            y_out[(int64_t)b * N + n] = acc;
+    for (int b = 0; b < B; ++b) {
+        double* y = y_out + (int64_t)b * N;
+        for (int n = 0; n < N; ++n) y[n] = 0.0;
+        for (int k = 0; k < K; ++k) {
+            const double ov = bf16_bits_to_double(o[(int64_t)b * K + k]);
+            const uint16_t* w = w_o + (int64_t)k * N;
+            for (int n = 0; n < N; ++n) y[n] += ov * bf16_bits_to_double(w[n]);
         }
     }
 }
