@@ -23,6 +23,8 @@ cudaError_t launch_qproj(const CUtensorMap& tw, const CUtensorMap& ta, const Qpr
                          int m_tiles, cudaStream_t stream);
 cudaError_t launch_kv_append(const CUtensorMap& twk, const CUtensorMap& twv, const CUtensorMap& tx,
                              const QprojParams& pg, const KvAppendParams& pm, cudaStream_t stream);
+cudaError_t launch_out_proj(const CUtensorMap& tw, const CUtensorMap& ta, const QprojParams& pg,
+                            __nv_bfloat16* y, int64_t y_stride, cudaStream_t stream);
 }  // namespace mfa
 
 using namespace mfa;
@@ -851,6 +853,76 @@ int mfa_kv_append(const mfa_tensor* x, const mfa_tensor* w_k, const mfa_tensor* 
 
   const cudaError_t e =
       launch_kv_append(twk, twv, tx, pg, pm, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MFA_OK : cuda_fail(e);
+}
+
+}  // extern "C"
+
+// ===========================================================================
+// Output projection
+// ===========================================================================
+namespace {
+
+// Split-K factor: the output's 128-feature tiles times this many k-ranges
+// cover the SMs at most once.
+int out_proj_splits(int64_t k, int64_t n, int sms) {
+  const int64_t tiles = n / 128;
+  int64_t s = tiles > 0 ? sms / tiles : 1;
+  if (s < 1) s = 1;
+  if (s > k / 64) s = k / 64;
+  return static_cast<int>(s);
+}
+
+size_t out_proj_ws_bytes(int64_t batch, int64_t k, int64_t n, int sms) {
+  return align256(static_cast<size_t>(out_proj_splits(k, n, sms)) * batch * n * sizeof(float));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mfa_output_proj_workspace_size(int batch, int k, int n) {
+  if (batch <= 0 || k <= 0 || n <= 0 || k % 64 || n % 128) return 0;
+  DeviceInfo d;
+  const int rc = current_device(&d);
+  if (rc != MFA_OK && rc != MFA_ERR_UNSUPPORTED) return 0;
+  return out_proj_ws_bytes(batch, k, n, d.sms);
+}
+
+int mfa_output_proj(const mfa_tensor* o, const mfa_tensor* w_o, mfa_tensor* y, void* workspace,
+                    size_t workspace_bytes, mfa_stream_t stream) {
+  if (!well_formed(o, 2) || !well_formed(w_o, 2) || !well_formed(y, 2)) return MFA_ERR_INVALID_ARG;
+  for (const mfa_tensor* t : std::initializer_list<const mfa_tensor*>{o, w_o, y})
+    if (t->dtype != MFA_BF16 || t->stride[1] != 1 || t->stride[0] % 8 || !aligned16(t->data))
+      return MFA_ERR_INVALID_ARG;
+  const int64_t B = o->shape[0], K = o->shape[1], N = w_o->shape[1];
+  if (w_o->shape[0] != K || y->shape[0] != B || y->shape[1] != N) return MFA_ERR_INVALID_ARG;
+  if (B < 1 || B > 256 || K <= 0 || K % 64 || K > (1 << 20) || N <= 0 || N % 128 ||
+      N > (1 << 20))
+    return MFA_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  int rc = current_device(&dev);
+  if (rc != MFA_OK) return rc;
+  if (!workspace || workspace_bytes < out_proj_ws_bytes(B, K, N, dev.sms) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return MFA_ERR_WORKSPACE;
+  const int n_cols = static_cast<int>((B + 15) / 16 * 16);
+  CUtensorMap tw, ta;
+  if (encode_2d(&tw, w_o->data, N, K, w_o->stride[0], 64, 64) != CUDA_SUCCESS ||
+      encode_2d(&ta, o->data, K, B, o->stride[0], 64, n_cols) != CUDA_SUCCESS)
+    return MFA_ERR_INVALID_ARG;
+  QprojParams pg;
+  std::memset(&pg, 0, sizeof pg);
+  pg.batch = static_cast<int>(B);
+  pg.k_blocks = static_cast<int>(K / 64);
+  pg.m_total = static_cast<int>(N);
+  pg.splits = out_proj_splits(K, N, dev.sms);
+  pg.n_cols = n_cols;
+  pg.mode = 2;
+  pg.partials = static_cast<float*>(workspace);
+  pg.m_half = static_cast<int>(N / 128);  // one weight map: every tile is the first's
+  const cudaError_t e = launch_out_proj(tw, ta, pg, static_cast<__nv_bfloat16*>(y->data),
+                                        y->stride[0], reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MFA_OK : cuda_fail(e);
 }
 

@@ -658,6 +658,59 @@ __global__ void __launch_bounds__(kMergeThreads)
   }
 }
 
+// ===========================================================================
+// Output projection y = o W_o: the GEMM above in mode 2 with one weight map
+// (split-K partials only), then a merge kernel in which a thread owns one
+// output element and sums the splits in order (deterministic) before one
+// rounding to bf16.
+// ===========================================================================
+__global__ void __launch_bounds__(kMergeThreads)
+    mfa_splitk_merge_kernel(const float* partials, int splits, int batch, int n,
+                            __nv_bfloat16* y, int64_t y_stride) {
+  griddep_wait();  // the partials of the projection kernel
+  const int64_t o = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
+  if (o >= static_cast<int64_t>(batch) * n) return;
+  const int b = static_cast<int>(o / n);
+  const int f = static_cast<int>(o % n);
+  float acc = 0.f;
+  for (int s0 = 0; s0 < splits; s0 += kAppendSplitBatch) {
+    float v[kAppendSplitBatch];
+#pragma unroll
+    for (int u = 0; u < kAppendSplitBatch; ++u)
+      v[u] = s0 + u < splits
+                 ? __ldcg(partials + (static_cast<int64_t>(s0 + u) * batch + b) * n + f)
+                 : 0.f;
+#pragma unroll
+    for (int u = 0; u < kAppendSplitBatch; ++u)
+      if (s0 + u < splits) acc += v[u];
+  }
+  y[static_cast<int64_t>(b) * y_stride + f] = __float2bfloat16_rn(acc);
+}
+
+cudaError_t launch_out_proj(const CUtensorMap& tw, const CUtensorMap& ta, const QprojParams& pg,
+                            __nv_bfloat16* y, int64_t y_stride, cudaStream_t stream) {
+  const int smem = qproj_smem_bytes(pg.n_cols);
+  cudaError_t err =
+      cudaFuncSetAttribute(mfa_qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  const int m_tiles = pg.m_total / 128;
+  mfa_qproj_kernel<<<dim3(m_tiles, pg.splits), kGemmThreads, smem, stream>>>(tw, ta, tw, pg);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t outputs = static_cast<int64_t>(pg.batch) * pg.m_total;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((outputs + kMergeThreads - 1) / kMergeThreads));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mfa_splitk_merge_kernel, static_cast<const float*>(pg.partials),
+                            pg.splits, pg.batch, pg.m_total, y, y_stride);
+}
+
 cudaError_t launch_kv_append(const CUtensorMap& twk, const CUtensorMap& twv, const CUtensorMap& tx,
                              const QprojParams& pg, const KvAppendParams& pm, cudaStream_t stream) {
   const int smem = qproj_smem_bytes(pg.n_cols);

@@ -177,6 +177,20 @@ def make_kv_append_inputs(seed: int, batch: int, hidden: int = HIDDEN) -> KvAppe
     return KvAppendInputs(x=x, w_k=w_k, w_v=w_v)
 
 
+@dataclass
+class OutProjInputs:
+    o: torch.Tensor    # [B, 64 * 256] bf16 attention outputs (heads x dim)
+    w_o: torch.Tensor  # [64 * 256, hidden] bf16
+
+
+def make_out_proj_inputs(seed: int, batch: int, hidden: int = HIDDEN) -> OutProjInputs:
+    """Attention outputs ~ N(0, 1) and W_o ~ N(0, 0.02), as the projection's weights."""
+    g = torch.Generator().manual_seed(int(seed))
+    o = _randn_bf16(g, (batch, H * D))
+    w_o = _randn_bf16(g, (H * D, hidden), std=0.02)
+    return OutProjInputs(o=o, w_o=w_o)
+
+
 # The five workloads (seed = 1000 + index). Index 2 is the headline workload.
 WORKLOADS = {
     1: dict(name="mfa_decode_b1_l512_bf16", batch=1, seq_len=512),

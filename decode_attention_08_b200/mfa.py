@@ -43,6 +43,7 @@ _lock = threading.Lock()
 EXPORTS = ("mfa_decode_attention", "mfa_decode_attention_ex", "mfa_decode_workspace_size",
            "mfa_query_proj", "mfa_query_proj_ex", "mfa_query_proj_workspace_size",
            "mfa_kv_append", "mfa_kv_append_workspace_size",
+           "mfa_output_proj", "mfa_output_proj_workspace_size",
            "mfa_read_status", "mfa_error_string", "mfa_version", "mfa_last_cuda_error_string",
            "mfa_decode_attention_noalloc")
 
@@ -81,6 +82,10 @@ def lib() -> ctypes.CDLL:
             L.mfa_kv_append.restype = ctypes.c_int
             L.mfa_kv_append_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int]
             L.mfa_kv_append_workspace_size.restype = ctypes.c_size_t
+            L.mfa_output_proj.argtypes = [T, T, T, P, ctypes.c_size_t, P]
+            L.mfa_output_proj.restype = ctypes.c_int
+            L.mfa_output_proj_workspace_size.argtypes = [ctypes.c_int] * 3
+            L.mfa_output_proj_workspace_size.restype = ctypes.c_size_t
             L.mfa_read_status.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
             L.mfa_read_status.restype = ctypes.c_int
             L.mfa_error_string.argtypes = [ctypes.c_int]
@@ -223,6 +228,23 @@ def kv_append(x, w_k, w_v, k_cache, v_cache, positions, page_table=None, kv_dtyp
                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "mfa_kv_append")
     return k_cache, v_cache
+
+
+def output_proj_workspace_size(batch: int, k: int, n: int) -> int:
+    return int(lib().mfa_output_proj_workspace_size(int(batch), int(k), int(n)))
+
+
+def output_proj(o, w_o, y, workspace=None, stream=None):
+    """``mfa_output_proj``: y = o W_o (o [B, K] = attention outputs, heads x dim)."""
+    if workspace is None:
+        n = output_proj_workspace_size(o.shape[0], o.shape[1], w_o.shape[1])
+        if n == 0:
+            raise RuntimeError("mfa_output_proj_workspace_size failed")
+        workspace = torch.empty(n, dtype=torch.uint8, device=o.device)
+    rc = lib().mfa_output_proj(describe(o), describe(w_o), describe(y), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mfa_output_proj")
+    return y
 
 
 def read_status(stream=None, reset: bool = True) -> int:

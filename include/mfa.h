@@ -228,6 +228,26 @@ int mfa_kv_append(const mfa_tensor* x, const mfa_tensor* w_k, const mfa_tensor* 
 
 size_t mfa_kv_append_workspace_size(int batch, int hidden);
 
+/*
+ * Output projection of the attention layer: y = o * W_o, o the attention
+ * outputs of each token with its 64 heads x 256 concatenated ([B, 16384] in
+ * Step-3, i.e. mfa_decode_attention's out viewed as [B, 64 * 256]), W_o
+ * [16384, 7168] bf16 row-major back to the hidden size, no bias. The pages name
+ * no W_o; this is the plain reading of an attention layer's output projection.
+ *
+ *  o    [B, K] bf16, w_o [K, N] bf16, y [B, N] bf16 (row strides multiples of 8).
+ *  workspace  at least mfa_output_proj_workspace_size(B, K, N) bytes, 256-byte
+ *             aligned, no initialisation needed (split-K partials).
+ * 1 <= B <= 256; K a multiple of 64, N of 128. fp32 accumulation split over K,
+ * partials summed in a fixed order, one rounding to bf16. Two kernels on `stream`.
+ * Returns MFA_OK, MFA_ERR_INVALID_ARG, MFA_ERR_UNSUPPORTED, MFA_ERR_WORKSPACE or
+ * MFA_ERR_CUDA.
+ */
+int mfa_output_proj(const mfa_tensor* o, const mfa_tensor* w_o, mfa_tensor* y, void* workspace,
+                    size_t workspace_bytes, mfa_stream_t stream);
+
+size_t mfa_output_proj_workspace_size(int batch, int k, int n);
+
 /* Synchronises `stream`, then reads (and, if reset != 0, clears) the current
  * device's status word: MFA_OK or the first MFA_ERR_BAD_INDEX / MFA_ERR_TIMEOUT
  * a kernel recorded since the last reset. Returns MFA_OK or MFA_ERR_CUDA. */

@@ -71,6 +71,7 @@ def test_null_and_malformed_descriptors_are_rejected_on_host(libmfa):
     assert libmfa.mfa_query_proj(null, null, null, null, None) == 1
     assert libmfa.mfa_kv_append(null, null, null, null, null, null, null, 0, 1.0, 1.0, None, 0,
                                 None) == 1
+    assert libmfa.mfa_output_proj(null, null, null, None, 0, None) == 1
 
 
 def _fake(shape, dtype_code, addr=0x100000, strides=None):
