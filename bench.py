@@ -413,6 +413,9 @@ def other_workloads(hbm_peak: float):
     for batch, kv in ((64, "bf16"), (128, "e4m3")):
         res[f"mfa_kv_append_b{batch}_h7168_{kv}"] = time_kv_append(batch, kv, hbm_peak)
         torch.cuda.empty_cache()
+    for batch in (8, 64):
+        res[f"mfa_output_proj_b{batch}_16384x7168"] = time_out_proj(batch, hbm_peak)
+        torch.cuda.empty_cache()
     return res
 
 
@@ -507,6 +510,47 @@ def time_kv_append(batch: int, kv_dtype: str, hbm_peak: float):
             "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak, "status": status,
             "note": "split-K projection x [W_k | W_v] (one launch) + merge-and-store kernel; "
                     "weights rotate through 20 copies (> L2)"}
+
+
+def time_out_proj(batch: int, hbm_peak: float):
+    """The attention layer's output projection [B, 16384] x [16384, 7168]; two
+    weight copies (235 MB each, > L2) alternate."""
+    from decode_attention_08_b200 import mfa
+    inp = gen.make_out_proj_inputs(4000 + batch, batch)
+    o = inp.o.cuda()
+    copies = [inp.w_o.cuda(), inp.w_o.cuda()]
+    y = torch.empty(batch, copies[0].shape[1], dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(mfa.output_proj_workspace_size(batch, o.shape[1], y.shape[1]),
+                     dtype=torch.uint8, device="cuda")
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        for i in range(3):
+            mfa.output_proj(o, copies[i % 2], y, workspace=ws, stream=st)
+    torch.cuda.synchronize()
+    graphs = []
+    for w in copies:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            mfa.output_proj(o, w, y, workspace=ws, stream=st)
+        graphs.append(g)
+    for i in range(4):
+        graphs[i % 2].replay()
+    torch.cuda.synchronize()
+    n = 50
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(st):
+        s.record(st)
+        for i in range(n):
+            graphs[i % 2].replay()
+        e.record(st)
+    torch.cuda.synchronize()
+    status = mfa.read_status()
+    t = s.elapsed_time(e) / 1e3 / n
+    alg = (copies[0].numel() + o.numel() + y.numel()) * 2
+    return {"us_per_call": t * 1e6, "alg_bytes": alg, "gbs": alg / t / 1e9,
+            "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak, "status": status,
+            "tflops": 2 * batch * copies[0].numel() / t / 1e12,
+            "note": "split-K GEMM (weights as the MMA's A operand) + in-order merge kernel"}
 
 
 def run_ours(args, world, rank, local):
