@@ -863,18 +863,18 @@ int mfa_kv_append(const mfa_tensor* x, const mfa_tensor* w_k, const mfa_tensor* 
 // ===========================================================================
 namespace {
 
-// Split-K factor: the output's 128-feature tiles times this many k-ranges
-// cover the SMs at most once.
-int out_proj_splits(int64_t k, int64_t n, int sms) {
-  const int64_t tiles = n / 128;
-  int64_t s = tiles > 0 ? sms / tiles : 1;
-  if (s < 1) s = 1;
-  if (s > k / 64) s = k / 64;
-  return static_cast<int>(s);
+// Stream-K grid: one CTA per SM, at least one per output tile (a CTA's run of
+// (tile, k-block) units then crosses at most one tile boundary).
+int out_proj_ctas(int64_t k, int64_t n, int sms) {
+  const int64_t tiles = n / 128, units = tiles * (k / 64);
+  int64_t g = sms < units ? sms : units;
+  if (g < tiles) g = tiles;
+  return static_cast<int>(g);
 }
 
+// Two fp32 partial slots [batch][128] per CTA.
 size_t out_proj_ws_bytes(int64_t batch, int64_t k, int64_t n, int sms) {
-  return align256(static_cast<size_t>(out_proj_splits(k, n, sms)) * batch * n * sizeof(float));
+  return align256(static_cast<size_t>(2) * out_proj_ctas(k, n, sms) * batch * 128 * sizeof(float));
 }
 
 }  // namespace
@@ -916,11 +916,9 @@ int mfa_output_proj(const mfa_tensor* o, const mfa_tensor* w_o, mfa_tensor* y, v
   pg.batch = static_cast<int>(B);
   pg.k_blocks = static_cast<int>(K / 64);
   pg.m_total = static_cast<int>(N);
-  pg.splits = out_proj_splits(K, N, dev.sms);
+  pg.splits = out_proj_ctas(K, N, dev.sms);  // the stream-K grid
   pg.n_cols = n_cols;
-  pg.mode = 2;
   pg.partials = static_cast<float*>(workspace);
-  pg.m_half = static_cast<int>(N / 128);  // one weight map: every tile is the first's
   const cudaError_t e = launch_out_proj(tw, ta, pg, static_cast<__nv_bfloat16*>(y->data),
                                         y->stride[0], reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MFA_OK : cuda_fail(e);

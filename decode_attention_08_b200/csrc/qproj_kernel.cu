@@ -659,30 +659,169 @@ __global__ void __launch_bounds__(kMergeThreads)
 }
 
 // ===========================================================================
-// Output projection y = o W_o: the GEMM above in mode 2 with one weight map
-// (split-K partials only), then a merge kernel in which a thread owns one
-// output element and sums the splits in order (deterministic) before one
-// rounding to bf16.
+// Output projection y = o W_o (stream-K GEMM + in-order merge, below).
 // ===========================================================================
+// ---------------------------------------------------------------------------
+// Stream-K output projection: the (tile, k-block) units, tile-major, are cut
+// into gridDim.x equal contiguous runs, one per CTA, so every SM streams the
+// same share of W_o (an even split per tile would leave SMs idle: 56 tiles).
+// A run crosses at most one tile boundary (tiles <= CTAs), so a CTA has one or
+// two segments, accumulated in two TMEM buffers; each segment's fp32 partial
+// goes to slot 2 * cta + segment. The merge sums, per output, the slots of the
+// CTAs whose runs cover its tile, in CTA order.
+// ---------------------------------------------------------------------------
+struct StreamKRun {
+  long long u0, u1;  // units [u0, u1) of this CTA
+};
+
+__host__ __device__ inline StreamKRun streamk_run(int cta, long long units, int ctas) {
+  return {static_cast<long long>(cta) * units / ctas,
+          static_cast<long long>(cta + 1) * units / ctas};
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mfa_streamk_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                            const __grid_constant__ CUtensorMap tm_act, const QprojParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int n_cols = p.n_cols;
+  const int stages = gemm_stages(n_cols);
+  const int stage_bytes = kABytes + n_cols * 128;
+  GemmCtrl& c = *reinterpret_cast<GemmCtrl*>(smem + stages * stage_bytes);
+  __shared__ uint64_t seg_ready[2];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int KB = p.k_blocks;
+  const long long units = static_cast<long long>(p.m_total / 128) * KB;
+  const StreamKRun run = streamk_run(blockIdx.x, units, gridDim.x);
+  const int nunits = static_cast<int>(run.u1 - run.u0);
+  // segment boundary: the first unit of the run's second tile (if any)
+  const long long split_u = (run.u0 / KB + 1) * KB;
+  const int nseg = nunits <= 0 ? 0 : (run.u1 > split_u ? 2 : 1);
+  const uint32_t tcols = gemm_tmem_cols(n_cols);
+
+  if (tid == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&c.full[i], 1);
+      mbar_init(&c.empty[i], 1);
+    }
+    mbar_init(&seg_ready[0], 1);
+    mbar_init(&seg_ready[1], 1);
+    c.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&c.tmem_base, 2 * tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  volatile int* abort_flag = &c.abort_flag;
+
+  if (warp == 0) {
+    // ---------------- producer: the whole warp, one elected lane issues ----------------
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_a = l2_policy_evict_last();
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_w);
+      tma_prefetch_desc(&tm_act);
+    }
+    __syncwarp();
+    int s = 0;
+    uint32_t ph = 0;
+    for (long long u = run.u0; u < run.u1; ++u) {
+      if (!mbar_wait_warp(&c.empty[s], ph ^ 1u, abort_flag)) break;
+      uint8_t* st = smem + s * stage_bytes;
+      const int tile = static_cast<int>(u / KB), kb = static_cast<int>(u % KB);
+      mbar_arrive_expect_tx_warp(&c.full[s], stage_bytes);
+      tma_load_2d_warp(st, &tm_w, &c.full[s], tile * 128, kb * 64, pol_w);
+      tma_load_2d_warp(st + kABytes / 2, &tm_w, &c.full[s], tile * 128 + 64, kb * 64, pol_w);
+      tma_load_2d_warp(st + kABytes, &tm_act, &c.full[s], kb * 64, 0, pol_a);
+      if (++s == stages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: the whole warp, one elected lane issues ----------------
+    const uint32_t idesc = idesc_f16(128, n_cols, 1, 1, 0);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (long long u = run.u0; u < run.u1 && ok; ++u) {
+      const int seg = u >= split_u ? 1 : 0;
+      const bool first = u == run.u0 || u == split_u;
+      if (!(ok = mbar_wait_warp(&c.full[s], ph, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t a = smem_u32(smem + s * stage_bytes);
+      const uint32_t b = a + kABytes;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_f16_ss_warp(tmem + seg * tcols, sw128_desc(a + k * 2048, kABytes / 2, 1024),
+                        sw128_desc(b + k * 32, 16, 1024), idesc, (!first || k > 0) ? 1u : 0u);
+      mma_commit_warp(&c.empty[s]);
+      if (u + 1 == run.u1 || u + 1 == split_u) mma_commit_warp(&seg_ready[seg]);
+      if (++s == stages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: thread = output feature row of the tile ----------------
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const int ml = warp * 32 + lane;
+  const int B = p.batch;
+  for (int seg = 0; seg < nseg; ++seg) {
+    const bool ready = mbar_wait(&seg_ready[seg], 0, abort_flag);
+    tc_fence_after();
+    if (!ready) break;
+    float* dst = p.partials + (static_cast<int64_t>(2 * blockIdx.x + seg) * B) * 128 + ml;
+    for (int cb = 0; cb < n_cols; cb += 16) {
+      uint32_t r[16];
+      tmem_ld16(taddr + seg * tcols + cb, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (cb + j < B) dst[static_cast<int64_t>(cb + j) * 128] = __uint_as_float(r[j]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 2 * tcols);
+}
+
+// The CTA whose run holds unit u (runs as in streamk_run).
+__device__ __forceinline__ int streamk_owner(long long u, long long units, int ctas) {
+  int c = static_cast<int>((u * ctas) / units);
+  while (c + 1 < ctas && streamk_run(c + 1, units, ctas).u0 <= u) ++c;
+  while (c > 0 && streamk_run(c, units, ctas).u0 > u) --c;
+  return c;
+}
+
 __global__ void __launch_bounds__(kMergeThreads)
-    mfa_splitk_merge_kernel(const float* partials, int splits, int batch, int n,
-                            __nv_bfloat16* y, int64_t y_stride) {
-  griddep_wait();  // the partials of the projection kernel
+    mfa_streamk_merge_kernel(const float* partials, int ctas, int k_blocks, int batch, int n,
+                             __nv_bfloat16* y, int64_t y_stride) {
+  griddep_wait();  // the partials of the stream-K kernel
   const int64_t o = static_cast<int64_t>(blockIdx.x) * kMergeThreads + threadIdx.x;
   if (o >= static_cast<int64_t>(batch) * n) return;
   const int b = static_cast<int>(o / n);
   const int f = static_cast<int>(o % n);
+  const int tile = f / 128, ml = f % 128;
+  const long long units = static_cast<long long>(n / 128) * k_blocks;
+  const long long t0 = static_cast<long long>(tile) * k_blocks;
+  const int c_lo = streamk_owner(t0, units, ctas);
+  const int c_hi = streamk_owner(t0 + k_blocks - 1, units, ctas);
   float acc = 0.f;
-  for (int s0 = 0; s0 < splits; s0 += kAppendSplitBatch) {
-    float v[kAppendSplitBatch];
-#pragma unroll
-    for (int u = 0; u < kAppendSplitBatch; ++u)
-      v[u] = s0 + u < splits
-                 ? __ldcg(partials + (static_cast<int64_t>(s0 + u) * batch + b) * n + f)
-                 : 0.f;
-#pragma unroll
-    for (int u = 0; u < kAppendSplitBatch; ++u)
-      if (s0 + u < splits) acc += v[u];
+  for (int cta = c_lo; cta <= c_hi; ++cta) {
+    // the segment of this CTA's run that lies in the tile: its second one if
+    // the run began in an earlier tile
+    const int seg = streamk_run(cta, units, ctas).u0 < t0 ? 1 : 0;
+    acc += __ldcg(partials + (static_cast<int64_t>(2 * cta + seg) * batch + b) * 128 + ml);
   }
   y[static_cast<int64_t>(b) * y_stride + f] = __float2bfloat16_rn(acc);
 }
@@ -693,8 +832,11 @@ cudaError_t launch_out_proj(const CUtensorMap& tw, const CUtensorMap& ta, const 
   cudaError_t err =
       cudaFuncSetAttribute(mfa_qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  const int m_tiles = pg.m_total / 128;
-  mfa_qproj_kernel<<<dim3(m_tiles, pg.splits), kGemmThreads, smem, stream>>>(tw, ta, tw, pg);
+  err = cudaFuncSetAttribute(mfa_streamk_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
+  if (err != cudaSuccess) return err;
+  // pg.splits carries the stream-K grid (CTAs, at least the number of tiles)
+  mfa_streamk_gemm_kernel<<<pg.splits, kGemmThreads, smem, stream>>>(tw, ta, pg);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int64_t outputs = static_cast<int64_t>(pg.batch) * pg.m_total;
@@ -707,8 +849,8 @@ cudaError_t launch_out_proj(const CUtensorMap& tw, const CUtensorMap& ta, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mfa_splitk_merge_kernel, static_cast<const float*>(pg.partials),
-                            pg.splits, pg.batch, pg.m_total, y, y_stride);
+  return cudaLaunchKernelEx(&cfg, mfa_streamk_merge_kernel, static_cast<const float*>(pg.partials),
+                            pg.splits, pg.k_blocks, pg.batch, pg.m_total, y, y_stride);
 }
 
 cudaError_t launch_kv_append(const CUtensorMap& twk, const CUtensorMap& twv, const CUtensorMap& tx,
