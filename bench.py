@@ -416,6 +416,9 @@ def other_workloads(hbm_peak: float):
     for batch in (8, 64):
         res[f"mfa_output_proj_b{batch}_16384x7168"] = time_out_proj(batch, hbm_peak)
         torch.cuda.empty_cache()
+    for batch in (8, 64):
+        res[f"mfa_lse_merge_b{batch}_s8"] = time_lse_merge(8, batch, hbm_peak)
+        torch.cuda.empty_cache()
     return res
 
 
@@ -551,6 +554,46 @@ def time_out_proj(batch: int, hbm_peak: float):
             "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak, "status": status,
             "tflops": 2 * batch * copies[0].numel() / t / 1e12,
             "note": "split-K GEMM (weights as the MMA's A operand) + in-order merge kernel"}
+
+
+def time_lse_merge(parts: int, batch: int, hbm_peak: float):
+    """The merge of a sequence split over `parts` GPUs (the exchange step's
+    compute): `parts` (O, lse) parts per sequence; enough input copies rotate
+    that the inputs exceed L2, one graph replays a call on each copy."""
+    from decode_attention_08_b200 import mfa
+    inp = gen.make_lse_merge_inputs(4100 + batch, parts, batch)
+    per_copy = (inp.o_parts.numel() + inp.lse_parts.numel()) * 4
+    n_copies = max(2, -(-2 * L2_BYTES // per_copy))
+    o_parts = [inp.o_parts.cuda() for _ in range(n_copies)]
+    lse_parts = [inp.lse_parts.cuda() for _ in range(n_copies)]
+    out = torch.empty(batch, 64, 256, dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        for i in range(3):
+            mfa.lse_merge(o_parts[i % n_copies], lse_parts[i % n_copies], out, stream=st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        for i in range(n_copies):
+            mfa.lse_merge(o_parts[i], lse_parts[i], out, stream=st)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = 5
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(st):
+        s.record(st)
+        for _ in range(reps):
+            g.replay()
+        e.record(st)
+    torch.cuda.synchronize()
+    status = mfa.read_status()
+    t = s.elapsed_time(e) / 1e3 / (reps * n_copies)
+    alg = per_copy + out.numel() * 2
+    return {"us_per_call": t * 1e6, "alg_bytes": alg, "gbs": alg / t / 1e9,
+            "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak, "status": status,
+            "copies": n_copies,
+            "note": "log-sum-exp merge of a sequence split over GPUs, bf16 output"}
 
 
 def run_ours(args, world, rank, local):

@@ -2,4 +2,5 @@
 // per-device status word needs no relocatable device code).
 #include "decode_kernel.cu"
 #include "qproj_kernel.cu"
+#include "merge_kernel.cu"
 #include "mfa_api.cu"

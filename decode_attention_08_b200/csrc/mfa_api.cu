@@ -25,6 +25,7 @@ cudaError_t launch_kv_append(const CUtensorMap& twk, const CUtensorMap& twv, con
                              const QprojParams& pg, const KvAppendParams& pm, cudaStream_t stream);
 cudaError_t launch_out_proj(const CUtensorMap& tw, const CUtensorMap& ta, const QprojParams& pg,
                             __nv_bfloat16* y, int64_t y_stride, cudaStream_t stream);
+cudaError_t launch_lse_merge(const LseMergeParams& p, cudaStream_t stream);
 }  // namespace mfa
 
 using namespace mfa;
@@ -925,3 +926,56 @@ int mfa_output_proj(const mfa_tensor* o, const mfa_tensor* w_o, mfa_tensor* y, v
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// log-sum-exp merge of partial results over disjoint key ranges
+// ---------------------------------------------------------------------------
+extern "C" int mfa_lse_merge(const mfa_tensor* o_parts, const mfa_tensor* lse_parts,
+                             mfa_tensor* out, mfa_tensor* lse_out, mfa_stream_t stream) {
+  if (!well_formed(o_parts, 4) || !well_formed(lse_parts, 3) || !well_formed(out, 3))
+    return MFA_ERR_INVALID_ARG;
+  if (o_parts->dtype != MFA_F32 || lse_parts->dtype != MFA_F32 ||
+      (out->dtype != MFA_BF16 && out->dtype != MFA_F32))
+    return MFA_ERR_INVALID_ARG;
+  const int64_t S = o_parts->shape[0], B = o_parts->shape[1];
+  if (S < 1 || S > (1 << 20) || B < 1 || B > (1 << 20)) return MFA_ERR_INVALID_ARG;
+  if (o_parts->shape[2] != kHeads || o_parts->shape[3] != kDim) return MFA_ERR_UNSUPPORTED;
+  if (lse_parts->shape[0] != S || lse_parts->shape[1] != B || lse_parts->shape[2] != kHeads ||
+      out->shape[0] != B || out->shape[1] != kHeads || out->shape[2] != kDim)
+    return MFA_ERR_INVALID_ARG;
+  // float4 loads of the parts; float4 (f32) or 8-byte (bf16) stores of the output
+  if (o_parts->stride[3] != 1 || o_parts->stride[2] % 4 || o_parts->stride[1] % 4 ||
+      o_parts->stride[0] % 4 || !aligned16(o_parts->data))
+    return MFA_ERR_INVALID_ARG;
+  if (lse_parts->stride[2] != 1) return MFA_ERR_INVALID_ARG;
+  const uintptr_t out_align = out->dtype == MFA_F32 ? 15u : 7u;
+  if (out->stride[2] != 1 || out->stride[1] % 4 || out->stride[0] % 4 ||
+      (reinterpret_cast<uintptr_t>(out->data) & out_align))
+    return MFA_ERR_INVALID_ARG;
+  if (lse_out && (!well_formed(lse_out, 2) || lse_out->dtype != MFA_F32 ||
+                  lse_out->shape[0] != B || lse_out->shape[1] != kHeads ||
+                  lse_out->stride[1] != 1))
+    return MFA_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  const int rc = current_device(&dev);
+  if (rc != MFA_OK) return rc;
+  LseMergeParams p;
+  std::memset(&p, 0, sizeof p);
+  p.o_parts = static_cast<const float*>(o_parts->data);
+  p.o_ss = o_parts->stride[0];
+  p.o_sb = o_parts->stride[1];
+  p.o_sh = o_parts->stride[2];
+  p.lse_parts = static_cast<const float*>(lse_parts->data);
+  p.l_ss = lse_parts->stride[0];
+  p.l_sb = lse_parts->stride[1];
+  p.parts = static_cast<int>(S);
+  p.batch = static_cast<int>(B);
+  p.out = out->data;
+  p.out_f32 = out->dtype == MFA_F32;
+  p.out_sb = out->stride[0];
+  p.out_sh = out->stride[1];
+  p.lse_out = lse_out ? static_cast<float*>(lse_out->data) : nullptr;
+  p.lse_sb = lse_out ? lse_out->stride[0] : 0;
+  const cudaError_t e = launch_lse_merge(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MFA_OK : cuda_fail(e);
+}

@@ -116,6 +116,20 @@ struct QprojFusedParams {
   int64_t q_stride;
 };
 
+// Log-sum-exp merge of attention results over disjoint key ranges.
+struct LseMergeParams {
+  const float* o_parts;  // [S][B][64][256], d stride 1
+  int64_t o_ss, o_sb, o_sh;
+  const float* lse_parts;  // [S][B][64], h stride 1
+  int64_t l_ss, l_sb;
+  int parts, batch;
+  void* out;  // [B][64][256] bf16 or f32, d stride 1
+  int out_f32;
+  int64_t out_sb, out_sh;
+  float* lse_out;  // nullable [B][64]
+  int64_t lse_sb;
+};
+
 constexpr int kQprojDone = 1023;  // counter index of the fused kernel's latent-ready count
 
 }  // namespace mfa

@@ -191,6 +191,27 @@ def make_out_proj_inputs(seed: int, batch: int, hidden: int = HIDDEN) -> OutProj
     return OutProjInputs(o=o, w_o=w_o)
 
 
+@dataclass
+class LseMergeInputs:
+    o_parts: torch.Tensor    # [S, B, 64, 256] float32
+    lse_parts: torch.Tensor  # [S, B, 64] float32, -inf marks an empty part
+
+
+def make_lse_merge_inputs(seed: int, parts: int, batch: int, empty: float = 0.0,
+                          lse_std: float = 4.0) -> LseMergeInputs:
+    """Parts of a log-sum-exp merge: outputs ~ N(0, 1), lse ~ N(0, lse_std); a
+    seeded fraction ``empty`` of the (part, sequence, head) entries is empty
+    (lse = -inf, its output NaN, which must not reach the result)."""
+    g = torch.Generator().manual_seed(int(seed))
+    o = torch.randn((parts, batch, H, D), generator=g, dtype=torch.float32)
+    lse = torch.randn((parts, batch, H), generator=g, dtype=torch.float32) * lse_std
+    if empty > 0:
+        hole = torch.rand((parts, batch, H), generator=g) < empty
+        lse[hole] = float("-inf")
+        o[hole] = float("nan")
+    return LseMergeInputs(o_parts=o, lse_parts=lse)
+
+
 # The five workloads (seed = 1000 + index). Index 2 is the headline workload.
 WORKLOADS = {
     1: dict(name="mfa_decode_b1_l512_bf16", batch=1, seq_len=512),

@@ -43,7 +43,7 @@ _lock = threading.Lock()
 EXPORTS = ("mfa_decode_attention", "mfa_decode_attention_ex", "mfa_decode_workspace_size",
            "mfa_query_proj", "mfa_query_proj_ex", "mfa_query_proj_workspace_size",
            "mfa_kv_append", "mfa_kv_append_workspace_size",
-           "mfa_output_proj", "mfa_output_proj_workspace_size",
+           "mfa_output_proj", "mfa_output_proj_workspace_size", "mfa_lse_merge",
            "mfa_read_status", "mfa_error_string", "mfa_version", "mfa_last_cuda_error_string",
            "mfa_decode_attention_noalloc")
 
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
             L.mfa_output_proj.restype = ctypes.c_int
             L.mfa_output_proj_workspace_size.argtypes = [ctypes.c_int] * 3
             L.mfa_output_proj_workspace_size.restype = ctypes.c_size_t
+            L.mfa_lse_merge.argtypes = [T, T, T, T, P]
+            L.mfa_lse_merge.restype = ctypes.c_int
             L.mfa_read_status.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
             L.mfa_read_status.restype = ctypes.c_int
             L.mfa_error_string.argtypes = [ctypes.c_int]
@@ -245,6 +247,15 @@ def output_proj(o, w_o, y, workspace=None, stream=None):
                                workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "mfa_output_proj")
     return y
+
+
+def lse_merge(o_parts, lse_parts, out, lse_out=None, stream=None):
+    """``mfa_lse_merge``: merge attention parts over disjoint key ranges
+    (o_parts [S, B, 64, 256] f32, lse_parts [S, B, 64] f32) into out [B, 64, 256]."""
+    rc = lib().mfa_lse_merge(describe(o_parts), describe(lse_parts), describe(out),
+                             describe(lse_out), _stream(stream))
+    _check(rc, "mfa_lse_merge")
+    return out
 
 
 def read_status(stream=None, reset: bool = True) -> int:

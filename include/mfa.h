@@ -248,6 +248,36 @@ int mfa_output_proj(const mfa_tensor* o, const mfa_tensor* w_o, mfa_tensor* y, v
 
 size_t mfa_output_proj_workspace_size(int batch, int k, int n);
 
+/*
+ * Log-sum-exp merge of attention results computed over disjoint key ranges of
+ * the same sequences (Flash-Decoding's combine, cited on the DeepSeek-V4 page's
+ * reference list). Part s holds, for each sequence b and head h, the output
+ * O_s[b,h,:] normalised over its own key range and that range's lse_s[b,h]
+ * (natural log; -inf for an empty range) -- exactly what mfa_decode_attention_ex
+ * returns in `out` (f32) and `lse_out` for the tokens it was given. The merge is
+ *
+ *     lse* = max_s lse_s,  w_s = exp(lse_s - lse*),
+ *     out[b,h,:] = sum_s w_s O_s[b,h,:] / sum_s w_s,  lse[b,h] = lse* + log sum_s w_s,
+ *
+ * i.e. the attention over the union of the ranges. It is the exchange step of a
+ * sequence whose cache is split across GPUs: each rank attends over its own
+ * range, the (O, lse) parts are gathered (NCCL), and the owner merges them here.
+ *
+ *  o_parts    [S, B, 64, 256] f32 (device), 16-byte aligned, all strides multiples of 4.
+ *  lse_parts  [S, B, 64] f32 (device), head stride 1. Values finite or -inf.
+ *  out        [B, 64, 256] bf16 (8-byte aligned) or f32 (16-byte aligned),
+ *             strides multiples of 4.
+ *  lse_out    [B, 64] f32 or NULL.
+ * 1 <= S <= 2^20, 1 <= B <= 2^20. Parts are merged in index order (results do
+ * not depend on timing). A part whose lse is -inf has no weight and its O is not
+ * used (it may hold anything); if every part of (b, h) is empty, out = 0 and
+ * lse = -inf, as for an empty sequence. One kernel on `stream`; out and lse_out
+ * must not overlap the parts. Returns MFA_OK, MFA_ERR_INVALID_ARG,
+ * MFA_ERR_UNSUPPORTED (head count or dim not 64 / 256; not a B200) or MFA_ERR_CUDA.
+ */
+int mfa_lse_merge(const mfa_tensor* o_parts, const mfa_tensor* lse_parts, mfa_tensor* out,
+                  mfa_tensor* lse_out, mfa_stream_t stream);
+
 /* Synchronises `stream`, then reads (and, if reset != 0, clears) the current
  * device's status word: MFA_OK or the first MFA_ERR_BAD_INDEX / MFA_ERR_TIMEOUT
  * a kernel recorded since the last reset. Returns MFA_OK or MFA_ERR_CUDA. */

@@ -72,6 +72,7 @@ def test_null_and_malformed_descriptors_are_rejected_on_host(libmfa):
     assert libmfa.mfa_kv_append(null, null, null, null, null, null, null, 0, 1.0, 1.0, None, 0,
                                 None) == 1
     assert libmfa.mfa_output_proj(null, null, null, None, 0, None) == 1
+    assert libmfa.mfa_lse_merge(null, null, null, null, None) == 1
 
 
 def _fake(shape, dtype_code, addr=0x100000, strides=None):
@@ -127,6 +128,26 @@ def test_shape_and_dtype_validation(libmfa):
     assert g(x, _fake([7000, 2048], 0), wb, qo, None) == 1
     assert g(_fake([129, 7168], 0), wa, wb, _fake([129, 16384], 0), None) == 2
     assert g(x, wa, wb, _fake([8, 16000], 0), None) == 1
+
+
+def test_lse_merge_validation(libmfa):
+    """Descriptor checks of mfa_lse_merge, before any CUDA call (fake addresses)."""
+    null = ctypes.POINTER(__import__("decode_attention_08_b200.mfa",
+                                     fromlist=["MfaTensor"]).MfaTensor)()
+    S, B = 4, 3
+    o = _fake([S, B, 64, 256], 1)
+    lse = _fake([S, B, 64], 1)
+    out = _fake([B, 64, 256], 0)
+    f = libmfa.mfa_lse_merge
+    assert f(_fake([S, B, 64, 256], 0), lse, out, null, None) == 1   # parts not f32
+    assert f(_fake([S, B, 32, 256], 1), lse, out, null, None) == 2   # 32 heads
+    assert f(o, _fake([S, B + 1, 64], 1), out, null, None) == 1      # lse shape
+    assert f(o, lse, _fake([B, 64, 256], 3), null, None) == 1        # out dtype
+    assert f(o, lse, out, _fake([B, 63], 1), None) == 1             # lse_out shape
+    assert f(_fake([0, B, 64, 256], 1), _fake([0, B, 64], 1), out, null, None) == 1  # no parts
+    misaligned = _fake([S, B, 64, 256], 1, strides=[B * 64 * 258, 64 * 258, 258, 1])
+    assert f(misaligned, lse, out, null, None) == 1                  # float4 loads need 16 B
+    assert f(o, lse, _fake([B, 64, 256], 0, addr=0x100004), null, None) == 1  # bf16 out 8 B
 
 
 def test_workspace_size_is_zero_for_bad_arguments(libmfa):
