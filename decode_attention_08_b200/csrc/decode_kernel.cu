@@ -1460,10 +1460,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
       // ---- per-head maximum over the tile's 128 rows --------------------
       {
-        float v[kWGHeads];
+        // per head, the maximum over this warp's 32 rows (every lane gets all
+        // 32); lane 0 hands them to the exchange
+        float r[kWGHeads];
 #pragma unroll
-        for (int h = 0; h < kWGHeads; ++h) v[h] = s[h];
-        c.red[g & 1][wg][sub][lane] = reduce_scatter32<true>(v, lane);
+        for (int h = 0; h < kWGHeads; ++h) r[h] = warp_max_f32(s[h]);
+        if (lane == 0) {
+          const uint32_t dst = smem_u32(&c.red[g & 1][wg][sub][0]);
+#pragma unroll
+          for (int q = 0; q < kWGHeads / 4; ++q)
+            st_shared_v4(dst + 16 * q, __float_as_uint(r[4 * q]), __float_as_uint(r[4 * q + 1]),
+                         __float_as_uint(r[4 * q + 2]), __float_as_uint(r[4 * q + 3]));
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.red_full[wg][g & 1]);
@@ -1484,6 +1492,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       __syncwarp();
 
       // ---- probabilities, row sums ---------------------------------------
+      if (rescale) {  // (rare) the row sums move to the new reference first
+#pragma unroll
+        for (int h = 0; h < kWGHeads; ++h) l_part[h] *= cv[h];
+      }
       uint32_t pk[kWGHeads / 2];
 #pragma unroll
       for (int h = 0; h < kWGHeads; h += 4) {
@@ -1492,18 +1504,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const float p1 = ex2_approx(s[h + 1] - m4.y);
         const float p2 = ex2_approx(s[h + 2] - m4.z);
         const float p3 = ex2_approx(s[h + 3] - m4.w);
-        if (rescale) {
-          const float4 c4 = *reinterpret_cast<const float4*>(&cv[h]);
-          l_part[h] = l_part[h] * c4.x + p0;
-          l_part[h + 1] = l_part[h + 1] * c4.y + p1;
-          l_part[h + 2] = l_part[h + 2] * c4.z + p2;
-          l_part[h + 3] = l_part[h + 3] * c4.w + p3;
-        } else {
-          l_part[h] += p0;
-          l_part[h + 1] += p1;
-          l_part[h + 2] += p2;
-          l_part[h + 3] += p3;
-        }
+        l_part[h] += p0;
+        l_part[h + 1] += p1;
+        l_part[h + 2] += p2;
+        l_part[h + 3] += p3;
         if (kFp8) {
           // E4M3 pairs: hi bytes of heads h..h+3 in pk[h / 4], lo bytes in pk[8 + h / 4]
           const uint32_t a = split_e4m3x2(p0, p1), b = split_e4m3x2(p2, p3);

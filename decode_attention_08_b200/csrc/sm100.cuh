@@ -489,6 +489,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Maximum of x over the 32 lanes of a converged warp, returned to every lane
+// (one redux.sync on f32, sm_100a).
+__device__ __forceinline__ float warp_max_f32(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
