@@ -50,7 +50,8 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle's CPU-baseline sample")
-    ap.add_argument("--profile", choices=["decode", "paged", "fp8", "qproj"], default=None,
+    ap.add_argument("--profile", choices=["decode", "paged", "fp8", "qproj", "lse_merge"],
+                    default=None,
                     help="profiling case for ncu: plain launches of one kernel family on a "
                          "reduced workload that still exceeds L2")
     return ap.parse_args()
@@ -707,7 +708,14 @@ def run_profile_case(args):
     from decode_attention_08_b200 import build, mfa
     build.build()
     torch.cuda.set_device(0)
-    if args.profile == "qproj":
+    if args.profile == "lse_merge":
+        # a sequence batch split over 8 GPUs: 8 parts x 256 sequences (134 MB > L2)
+        inp = gen.make_lse_merge_inputs(4200, 8, 256)
+        o, l = inp.o_parts.cuda(), inp.lse_parts.cuda()
+        out = torch.empty(256, 64, 256, dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            mfa.lse_merge(o, l, out)
+    elif args.profile == "qproj":
         proj = gen.make_proj_inputs(2005, 8)
         x, wa, wb = proj.x.cuda(), proj.w_qa.cuda(), proj.w_qb.cuda()
         q = torch.empty(8, wb.shape[1], dtype=torch.bfloat16, device="cuda")

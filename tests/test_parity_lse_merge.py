@@ -142,3 +142,40 @@ def test_sequence_split_over_ranks_equals_whole(world, kv_dtype):
     assert mfa.read_status() == 0
     diff = (whole - out).abs().max().item()
     assert diff <= (3e-2 if kv_dtype == "e4m3" else 2e-3), diff
+
+
+def test_sharded_decode_through_a_process_group():
+    """seqshard.sharded_decode end to end on one GPU: a one-rank NCCL group (the
+    all-gather then holds this rank's part only), so the call must equal the
+    oracle over the whole sequences."""
+    import datetime
+    import os
+    import socket
+
+    import torch.distributed as dist
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        lens = [1000, 129]
+        dec = gen.make_decode_inputs(650, len(lens), lens)
+        k, v, n = _local_cache(dec, 0, 1)
+        out = torch.full((len(lens), 64, 256), float("nan"), device="cuda")
+        lse = torch.full((len(lens), 64), float("nan"), device="cuda")
+        seqshard.sharded_decode(dec.q.cuda(), k, v, n, out, softmax_scale=dec.softmax_scale,
+                                lse_out=lse)
+        assert mfa.read_status() == 0
+        pairs = sample_pairs(len(lens), 24, 8)
+        ref, ref_lse = oracle_decode(dec, select=pairs)
+        bi = [b for b, _ in pairs]
+        hi = [h for _, h in pairs]
+        got = out.double().cpu().numpy()[bi, hi]
+        assert_close(got, ref, decode_atol(dec, ref, torch.float32, b_index=bi), "sharded")
+        assert_close(lse.double().cpu().numpy()[bi, hi], ref_lse,
+                     1e-4 + 1e-5 * np.abs(ref_lse), "sharded lse")
+    finally:
+        dist.destroy_process_group()
