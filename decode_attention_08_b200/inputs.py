@@ -212,6 +212,93 @@ def make_lse_merge_inputs(seed: int, parts: int, batch: int, empty: float = 0.0,
     return LseMergeInputs(o_parts=o, lse_parts=lse)
 
 
+# Grouped-query comparison shape (the Step-3 summary page, "Key points ->
+# Ablations", compares MFA's decode latency with GQA's): 64 query heads of
+# dimension 128 in 2 groups of 32, each group with its own key and value head
+# of dimension 128, so a cached token costs 2 x 2 x 128 x 2 B = 1024 B, the same
+# as MFA's one 256-wide key head and value head.
+GQA_HEADS = 64
+GQA_GROUPS = 2
+GQA_DIM = 128
+
+
+@dataclass
+class GqaInputs:
+    q: torch.Tensor                  # [B, 64, 128] bf16
+    k: torch.Tensor                  # contiguous [B, Lmax, 2, 128] or paged [P, page, 2, 128]; bf16
+    v: torch.Tensor
+    seq_lens: torch.Tensor           # [B] int32
+    page_table: Optional[torch.Tensor] = None
+    page_size: int = 0
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def batch(self) -> int:
+        return self.q.shape[0]
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(GQA_DIM)
+
+    @property
+    def total_tokens(self) -> int:
+        return int(self.seq_lens.sum())
+
+
+def make_gqa_inputs(seed: int, batch: int, seq_lens, *, lmax: Optional[int] = None,
+                    page_size: int = 0) -> GqaInputs:
+    """One grouped-query problem, drawn like make_decode_inputs (q, K, V ~ N(0, 1)
+    in bf16, seeded page placement, rows past a sequence's length NaN)."""
+    g = torch.Generator().manual_seed(int(seed))
+    if isinstance(seq_lens, int):
+        lens = torch.full((batch,), seq_lens, dtype=torch.int32)
+    else:
+        lens = torch.as_tensor(list(seq_lens), dtype=torch.int32)
+    assert lens.numel() == batch
+    q = _randn_bf16(g, (batch, GQA_HEADS, GQA_DIM))
+    pt = None
+    if page_size > 0:
+        pages_per_seq = [(int(L) + page_size - 1) // page_size for L in lens.tolist()]
+        pool = sum(pages_per_seq)
+        max_pages = max([1] + pages_per_seq)
+        perm = torch.randperm(max(pool, 1), generator=g)[:pool]
+        pt = torch.full((batch, max_pages), -1, dtype=torch.int32)
+        idx = 0
+        for b, n in enumerate(pages_per_seq):
+            if n:
+                pt[b, :n] = perm[idx: idx + n].to(torch.int32)
+            idx += n
+        shape = (max(pool, 1), page_size, GQA_GROUPS, GQA_DIM)
+    else:
+        L = int(lmax if lmax is not None else max([1] + lens.tolist()))
+        shape = (batch, L, GQA_GROUPS, GQA_DIM)
+    k = _randn_bf16(g, shape)
+    v = _randn_bf16(g, shape)
+    for b, L in enumerate(lens.tolist()):
+        if page_size > 0:
+            n = (L + page_size - 1) // page_size
+            if n and L % page_size:
+                last = int(pt[b, n - 1])
+                k[last, L % page_size:] = float("nan")
+                v[last, L % page_size:] = float("nan")
+        elif L < shape[1]:
+            k[b, L:] = float("nan")
+            v[b, L:] = float("nan")
+    return GqaInputs(q=q, k=k, v=v, seq_lens=lens, page_table=pt, page_size=page_size,
+                     meta={"seed": seed})
+
+
+GQA_WORKLOAD = dict(name="gqa_decode_b64_l4096_g2x128_bf16", batch=64, seq_len=4096)
+
+
+def make_gqa_workload() -> GqaInputs:
+    """The grouped-query comparison workload at the headline's size and bytes."""
+    w = GQA_WORKLOAD
+    inp = make_gqa_inputs(1100, w["batch"], w["seq_len"])
+    inp.meta.update(name=w["name"])
+    return inp
+
+
 # The five workloads (seed = 1000 + index). Index 2 is the headline workload.
 WORKLOADS = {
     1: dict(name="mfa_decode_b1_l512_bf16", batch=1, seq_len=512),

@@ -163,6 +163,78 @@ int mfa_oracle_decode(int B, int H, int D, const uint16_t* q,
 }
 
 /*
+ * Grouped-query attention (GQA; Ainslie et al., cited in the pages' reference
+ * lists; the Step-3 summary page, "Key points -> Ablations", compares MFA with
+ * it): H query heads of dimension D in G groups of H / G consecutive heads;
+ * group g has its own key head and value head of dimension D, so a cached token
+ * holds G key rows and G value rows. Head h belongs to group g = h / (H / G):
+ *
+ *     s[t]      = scale * sum_i q[b,h,i] * K_b[t,g,i]                 (t < L_b)
+ *     out[b,h,:] = sum_t softmax(s)[t] * V_b[t,g,:],   lse as for MFA above
+ *
+ * q: [B][H][D] bf16 bits. k, v: bf16 bits, contiguous [B][Lmax][G][D] (strides
+ * batch_stride, token_stride in elements; a token's G rows adjacent) or paged
+ * [num_pages][page_size][G][D] through the page table. out [B][H][D], lse
+ * [B][H]. Empty sequences: zeros, -inf. Returns 0, or -1 on an out-of-range page
+ * id / bad argument.
+ */
+int mfa_oracle_gqa_decode(int B, int H, int G, int D, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, int64_t batch_stride, int64_t token_stride,
+                          const int32_t* page_table, int max_pages, int page_size, int num_pages,
+                          const int32_t* seq_lens, double scale, double* out, double* lse) {
+    int bad = 0;
+    if (B < 0 || H <= 0 || G <= 0 || D <= 0 || H % G != 0) return -1;
+    const int heads_per_group = H / G;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int p = 0; p < B * H; ++p) {
+        int b = p / H, h = p % H;
+        int g = h / heads_per_group;
+        double* o = out + (int64_t)p * D;
+        int L = seq_lens[b];
+        if (L <= 0) {
+            for (int i = 0; i < D; ++i) o[i] = 0.0;
+            lse[p] = -INFINITY;
+            continue;
+        }
+        double* s = (double*)malloc(sizeof(double) * (size_t)L);
+        int64_t* row = (int64_t*)malloc(sizeof(int64_t) * (size_t)L);
+        /* element index of K_b[t][g][0] (same for V) */
+        for (int t = 0; t < L; ++t) {
+            if (page_table) {
+                int32_t phys = page_table[(int64_t)b * max_pages + t / page_size];
+                if (phys < 0 || phys >= num_pages) { bad = 1; row[t] = -1; continue; }
+                row[t] = (((int64_t)phys * page_size + t % page_size) * G + g) * D;
+            } else {
+                row[t] = (int64_t)b * batch_stride + (int64_t)t * token_stride + (int64_t)g * D;
+            }
+        }
+        double smax = -INFINITY;
+        for (int t = 0; t < L; ++t) {
+            double acc = 0.0;
+            if (row[t] >= 0)
+                for (int i = 0; i < D; ++i)
+                    acc += bf16_bits_to_double(q[((int64_t)b * H + h) * D + i]) *
+                           bf16_bits_to_double(k[row[t] + i]);
+            s[t] = scale * acc;
+            if (s[t] > smax) smax = s[t];
+        }
+        double denom = 0.0;
+        for (int t = 0; t < L; ++t) denom += exp(s[t] - smax);
+        for (int i = 0; i < D; ++i) o[i] = 0.0;
+        for (int t = 0; t < L; ++t) {
+            double w = exp(s[t] - smax) / denom;
+            if (row[t] >= 0)
+                for (int i = 0; i < D; ++i) o[i] += w * bf16_bits_to_double(v[row[t] + i]);
+        }
+        lse[p] = smax + log(denom);
+        free(s);
+        free(row);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
  * Split-KV merge (Flash-Decoding, cited on the DeepSeek-V4 page): n partial
  * results of the same softmax over disjoint token ranges, each normalised within
  * its own range and carrying its range's log-sum-exp, merge into the result over

@@ -76,6 +76,32 @@ def decode(q_bits, k, v, seq_lens, scale, *, kv_dtype=0, page_table=None, page_s
     return out, lse
 
 
+def gqa_decode(q_bits, k, v, seq_lens, scale, *, page_table=None, page_size=64):
+    """Grouped-query attention: q [B, H, D] bf16 bits, caches [.., G, D] bf16 bits;
+    the H heads form G consecutive groups, group g attends over key/value head g.
+    Returns out [B, H, D], lse [B, H]."""
+    q = bf16_bits_to_f64(q_bits)
+    B, H, D = q.shape
+    kd, vd = bf16_bits_to_f64(k), bf16_bits_to_f64(v)
+    G = kd.shape[-2]
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.full((B, H), -np.inf)
+    for b in range(B):
+        L = int(seq_lens[b])
+        if L <= 0:
+            continue
+        Kb = gather_sequence(kd, b, L, page_table, page_size)     # [L, G, D]
+        Vb = gather_sequence(vd, b, L, page_table, page_size)
+        qg = q[b].reshape(G, H // G, D)                           # [G, H/G, D]
+        s = scale * np.einsum("gjd,tgd->gjt", qg, Kb)             # [G, H/G, L]
+        m = s.max(axis=2, keepdims=True)
+        e = np.exp(s - m)
+        denom = e.sum(axis=2, keepdims=True)
+        out[b] = np.einsum("gjt,tgd->gjd", e / denom, Vb).reshape(H, D)
+        lse[b] = (m + np.log(denom)).reshape(H)
+    return out, lse
+
+
 def combine(parts, part_lse):
     """Flash-Decoding merge of per-range normalised partials."""
     parts = np.asarray(parts, np.float64)

@@ -62,6 +62,10 @@ def _load():
             lib.mfa_oracle_e4m3_encode.argtypes = [ctypes.c_double]
             lib.mfa_oracle_out_proj.restype = None
             lib.mfa_oracle_out_proj.argtypes = [ctypes.c_int] * 3 + [P, P, P]
+            lib.mfa_oracle_gqa_decode.restype = ctypes.c_int
+            lib.mfa_oracle_gqa_decode.argtypes = [
+                ctypes.c_int] * 4 + [P, P, P, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int, P, ctypes.c_double, P, P]
             lib.mfa_oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -127,6 +131,40 @@ def decode(q_bits, k, v, seq_lens, scale, *, kv_dtype=BF16, page_table=None, pag
                                _ptr(page_table), max_pages, psize, num_pages, _ptr(seq_lens),
                                float(scale), float(k_scale), float(v_scale), _ptr(sel_b),
                                _ptr(sel_h), n, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle: out-of-range page id or bad argument")
+    return out, lse
+
+
+def gqa_decode(q_bits, k, v, seq_lens, scale, *, page_table=None, page_size=64):
+    """Grouped-query decode attention in float64 (bf16 inputs).
+
+    q_bits: uint16 [B, H, D]. k, v: uint16 contiguous [B, Lmax, G, D] or, with
+    ``page_table``, paged [num_pages, page_size, G, D]. Head h uses group
+    h // (H // G). Returns (out [B, H, D], lse [B, H]) float64.
+    """
+    lib = _load()
+    q_bits = _c(q_bits, np.uint16)
+    B, H, D = q_bits.shape
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    assert k.shape == v.shape and k.shape[-1] == D and k.ndim == 4
+    G = k.shape[2]
+    seq_lens = _c(seq_lens, np.int32)
+    if page_table is not None:
+        page_table = _c(page_table, np.int32)
+        num_pages, psize = k.shape[0], k.shape[1]
+        assert psize == page_size
+        max_pages = page_table.shape[1]
+        bstride, tstride = 0, 0
+    else:
+        num_pages, max_pages, psize = 0, 0, 0
+        bstride, tstride = k.shape[1] * G * D, G * D
+    out = np.zeros((B, H, D), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    rc = lib.mfa_oracle_gqa_decode(B, H, G, D, _ptr(q_bits), _ptr(k), _ptr(v), bstride, tstride,
+                                   _ptr(page_table), max_pages, psize, num_pages,
+                                   _ptr(seq_lens), float(scale), _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle: out-of-range page id or bad argument")
     return out, lse
