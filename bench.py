@@ -41,7 +41,7 @@ UNIT = "KV-tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
@@ -54,23 +54,53 @@ def parse_args():
                     default=None,
                     help="profiling case for ncu: plain launches of one kernel family on a "
                          "reduced workload that still exceeds L2")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
 def dist_setup(gpus: int):
+    """Join the job's process group (one rank per GPU; NCCL, or gloo without
+    CUDA) from the rendezvous environment torchrun or spawn_ranks sets."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl" if torch.cuda.is_available() else "gloo",
+            timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
+
+
+def _free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _spawned_rank(local, world, port, target, target_args):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(local),
+                      LOCAL_RANK=str(local), WORLD_SIZE=str(world), LOCAL_WORLD_SIZE=str(world))
+    os.environ.setdefault("NCCL_DEBUG", "INFO")        # NCCL's init lines show the rank count
+    os.environ.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+    target(*target_args)
+
+
+def spawn_ranks(n: int, target, *target_args):
+    """Run target(*target_args) in n fresh processes, rank r on GPU r, with the
+    rendezvous environment torchrun would set (127.0.0.1, a free port): what
+    `bench.py --gpus N` does when it is not already running under torchrun."""
+    import torch.multiprocessing as mp
+    mp.spawn(_spawned_rank, args=(n, _free_port(), target, target_args), nprocs=n, join=True)
 
 
 def _dist_device() -> str:
@@ -284,6 +314,24 @@ def time_steps(step: DecodeStep, k: int, world: int):
     return s.elapsed_time(e) / 1e3
 
 
+def single_call_us(step: DecodeStep, n: int = 30) -> float:
+    """Latency of one call with nothing overlapping it: each replay of a
+    one-call graph (cache copies rotating) sits between two synchronisations;
+    the median device time between CUDA events on its stream, in us."""
+    times = []
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    for i in range(n):
+        torch.cuda.synchronize()
+        with torch.cuda.stream(step.stream):
+            s.record(step.stream)
+            step.replay(i)
+            e.record(step.stream)
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e) * 1e3)
+    return statistics.median(times)
+
+
 def sustain(step: DecodeStep, seconds: float):
     """Untimed load so the clock samples reflect the steady state."""
     t0 = time.time()
@@ -372,6 +420,18 @@ def e2e_decode(dec: gen.DecodeInputs, step: DecodeStep, k: int, world: int):
     return t, h2d, d2h
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (/proc/cpuinfo), for the CPU-baseline record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(dec: gen.DecodeInputs, seconds: float):
     """The float64 oracle on whole sequences of the same workload, until about
     `seconds` of CPU work; KV-tokens/s over the sample."""
@@ -392,14 +452,17 @@ def cpu_baseline(dec: gen.DecodeInputs, seconds: float):
         nseq += 1
         b += 1
     t = time.time() - t0
-    return {"value": done_tokens / t, "unit": UNIT, "cores": orc.num_threads(), "kind": "oracle",
+    return {"value": done_tokens / t, "unit": UNIT, "cores": orc.num_threads(), "cpu": cpu_model(),
+            "kind": "oracle",
             "sample": f"{nseq} of {dec.batch} sequences (all 64 heads, L=4096 each) of the "
                       f"headline workload, float64 C oracle, {t:.1f} s"}
 
 
-def other_workloads(hbm_peak: float):
+def other_workloads(hbm_peak: float, mfa_us: float):
     """Kernel-level numbers of the other workloads (one call per replay)."""
     res = {}
+    res[gen.GQA_WORKLOAD["name"]] = time_gqa(hbm_peak, mfa_us)
+    torch.cuda.empty_cache()
     for idx in (1, 3, 4, 5):
         dec, proj = gen.make_workload(idx)
         big = decode_alg_bytes(dec) > L2_BYTES
@@ -413,7 +476,8 @@ def other_workloads(hbm_peak: float):
         t = time_steps(step, n, 1) / n
         alg = decode_alg_bytes(dec)
         err, ns = spot_parity(dec, step.out)
-        entry = {"us_per_call": t * 1e6, "kv_tokens_per_s": dec.total_tokens / t,
+        entry = {"us_per_call": t * 1e6, "single_call_us": single_call_us(step),
+                 "kv_tokens_per_s": dec.total_tokens / t,
                  "seq_per_s": dec.batch / t, "alg_bytes": alg, "gbs": alg / t / 1e9,
                  "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak,
                  "spot_max_abs_err": err, "spot_samples": ns,
@@ -430,6 +494,9 @@ def other_workloads(hbm_peak: float):
             del step0
         if proj is not None:
             entry["qproj"] = time_qproj(proj, hbm_peak)
+            torch.cuda.empty_cache()
+            entry["fused_qproj_attention"] = time_fused(dec, proj, hbm_peak, t * 1e6,
+                                                        entry["qproj"]["us_per_call"])
         res[gen.WORKLOADS[idx]["name"]] = entry
         del step
         torch.cuda.empty_cache()
@@ -442,6 +509,89 @@ def other_workloads(hbm_peak: float):
     for batch in (8, 64):
         res[f"mfa_lse_merge_b{batch}_s8"] = time_lse_merge(8, batch, hbm_peak)
         torch.cuda.empty_cache()
+    return res
+
+
+class GqaStep(DecodeStep):
+    """DecodeStep over the grouped-query comparison kernel (same rotation and graphs)."""
+
+    def __init__(self, inp: gen.GqaInputs, copies: int):
+        from decode_attention_08_b200 import mfa
+        self.mfa = mfa
+        self.dec = inp
+        self.q = inp.q.cuda()
+        self.lens = inp.seq_lens.cuda()
+        self.pt = None
+        self.kv = [(inp.k.cuda(), inp.v.cuda()) for _ in range(copies)]
+        self.out = torch.empty(inp.batch, 64, 128, dtype=torch.bfloat16, device="cuda")
+        self.num_splits = 0
+        self.ws = torch.empty(mfa.decode_workspace_size(inp.batch, 0), dtype=torch.uint8,
+                              device="cuda")
+        self.graphs = []
+        self.stream = torch.cuda.Stream()
+
+    def call(self, i: int):
+        k, v = self.kv[i % len(self.kv)]
+        self.mfa.gqa_decode_attention(self.q, k, v, None, self.lens, self.out,
+                                      self.dec.softmax_scale, workspace=self.ws)
+
+
+def time_gqa(hbm_peak: float, mfa_us: float):
+    """The grouped-query comparison workload (same batch, context and cache bytes
+    per token as the headline), timed like the headline."""
+    inp = gen.make_gqa_workload()
+    step = GqaStep(inp, copies=3)
+    step.capture()
+    for i in range(5):
+        step.replay(i)
+    n = 200
+    t = time_steps(step, n, 1) / n
+    T = inp.total_tokens
+    alg = T * 1024 + inp.batch * 64 * 128 * 4 + inp.batch * 4
+    return {"us_per_call": t * 1e6, "single_call_us": single_call_us(step),
+            "kv_tokens_per_s": T / t, "alg_bytes": alg, "gbs": alg / t / 1e9,
+            "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak,
+            "mfa_headline_us_per_call": mfa_us, "gqa_over_mfa_time": t * 1e6 / mfa_us,
+            "shape": "64 q heads x 128 in 2 groups, 2 key + 2 value heads x 128 (1024 B/token, "
+                     "as MFA's 1 + 1 heads x 256), bf16 cache and output",
+            "l2": "3 rotating device copies of the cache"}
+
+
+class FusedStep(DecodeStep):
+    """The query projection then the attention in one call (mfa_qproj_decode_attention)."""
+
+    def __init__(self, dec: gen.DecodeInputs, proj: gen.ProjInputs, copies: int, num_splits: int):
+        super().__init__(dec, copies, num_splits=num_splits)
+        mfa = self.mfa
+        self.x, self.wa, self.wb = proj.x.cuda(), proj.w_qa.cuda(), proj.w_qb.cuda()
+        self.qf = torch.empty(dec.batch, 64 * 256, dtype=torch.bfloat16, device="cuda")
+        self.wsf = torch.zeros(mfa.qproj_decode_workspace_size(dec.batch, self.x.shape[1],
+                                                               self.wa.shape[1], num_splits),
+                               dtype=torch.uint8, device="cuda")
+
+    def call(self, i: int):
+        k, v = self.kv[i % len(self.kv)]
+        self.mfa.qproj_decode_attention(self.x, self.wa, self.wb, self.qf, k, v, self.pt,
+                                        self.lens, self.out, self.dec.softmax_scale,
+                                        num_splits=self.num_splits, workspace=self.wsf)
+
+
+def time_fused(dec: gen.DecodeInputs, proj: gen.ProjInputs, hbm_peak: float, attn_us: float,
+               proj_us: float):
+    """Projection + attention as one call, against the two timed separately."""
+    step = FusedStep(dec, proj, 2, dec.meta.get("num_splits", 0))
+    step.capture()
+    for i in range(5):
+        step.replay(i)
+    n = 50
+    t = time_steps(step, n, 1) / n
+    alg = decode_alg_bytes(dec) + sum(x.numel() * 2 for x in (proj.x, proj.w_qa, proj.w_qb))
+    res = {"us_per_call": t * 1e6, "single_call_us": single_call_us(step),
+           "sum_of_separate_us": attn_us + proj_us, "alg_bytes": alg, "gbs": alg / t / 1e9,
+           "frac_of_measured_hbm": alg / t / 1e9 / hbm_peak,
+           "note": "mfa_qproj_decode_attention: x[8,7168] -> W_qa -> W_qb -> q, then the 16-way "
+                   "split attention; algorithmic bytes = weights + x + the attention's"}
+    del step
     return res
 
 
@@ -667,6 +817,9 @@ def run_ours(args, world, rank, local):
         "clocks": clocks,
         "gpu_launches": 2 * args.steps,
     }
+    # one isolated call (nothing before or after it on the GPU) next to the
+    # pipelined per-step time above
+    line["single_call_us"] = single_call_us(step)
     if rank == 0:
         err, ns = spot_parity(dec, step.out)
         line["parity"] = {"spot_max_abs_err": err, "samples": ns, "tol": 2e-3}
@@ -683,7 +836,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_extra:
         del step
         torch.cuda.empty_cache()
-        line["other_workloads"] = other_workloads(hbm_peak)
+        line["other_workloads"] = other_workloads(hbm_peak, per_launch * 1e6)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -717,7 +870,7 @@ def run_reference(args, world, rank):
         "data": "synthetic (seeded N(0,1) q/K/V, bf16)", "impl": "reference",
         "config": {"workload": gen.WORKLOADS[HEADLINE]["name"], "batch_per_gpu": dec.batch,
                    "seq_len": 4096, "q_heads": 64, "head_dim": 256, "kv_heads": 1},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.num_threads(),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.num_threads(), "cpu": cpu_model(),
                          "kind": "oracle",
                          "sample": "per step one sequence (all 64 heads, L=4096) of the "
                                    "headline workload, float64 C oracle"},
@@ -761,8 +914,10 @@ def run_profile_case(args):
                       "status": mfa.read_status()}))
 
 
-def main():
-    args = parse_args()
+def main(argv=None, runner=None):
+    """Entry point. `runner(args, world, rank, local)` runs one rank's work
+    (default: the benchmark itself)."""
+    args = parse_args(argv)
     if args.profile:
         run_profile_case(args)
         return
@@ -770,9 +925,13 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
         return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # launch one rank per GPU ourselves (under torchrun they already exist)
+        spawn_ranks(args.gpus, main, sys.argv[1:] if argv is None else list(argv), runner)
+        return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_ours(args, world, rank, local)
+        (runner or run_ours)(args, world, rank, local)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

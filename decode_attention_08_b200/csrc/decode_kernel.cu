@@ -1,4 +1,4 @@
-// decode_kernel.cu -- MFA decode attention on sm_100a (bf16 KV cache).
+// decode_kernel.cu -- MFA decode attention on sm_100a (bf16 or FP8 E4M3 KV cache).
 //
 // Step-3 page, "Key points -> Architecture": the 64 query heads of a token all
 // attend over ONE shared key head and ONE shared value head of dimension 256.
@@ -6,18 +6,23 @@
 // attention are dense contractions and run on the 5th-generation tensor core:
 //
 //   S^T[t, h] = sum_i K[t, i] * q[h, i]       M = 128 tokens, N = 64 heads, K = 256
-//   O^T[i, h] += sum_t V[t, i] * P[h, t]      M = 128 dims (x2), N = 64 heads, K = 128 tokens
+//   O^T[i, h] += sum_t V[t, i] * P[h, t]      M = 128 dims (x2), N = 64 heads x (hi, lo), K = 128 tokens
 //
 // Both are issued "swap-AB" (tokens / head dims on the MMA's M side) so every
 // accumulator uses the M = 128 TMEM layout where TMEM lane = matrix row. The
 // softmax is computed online over 128-token tiles (running max with lazy
 // rescaling, running sum), so each K and V row is read from HBM exactly once.
+// The probabilities enter the PV product as an exact-sum pair hi + lo (bf16
+// pair, or E4M3 pair with an FP8 cache) in one N = 128 product per step.
 //
 // CTA = 12 warps, one CTA per SM (persistent):
-//   warp 0       TMA producer for the K/V ring (5 slots x 32 KB)
-//   warp 1       TMEM allocator + tcgen05.mma issuer (one lane issues)
-//   warp 2       TMA producer for q (one 32 KB load per sequence segment)
-//   warp 3       idle
+//   warp 0       TMA producer for the K/V ring (4 slots x 32 KB)
+//   warp 1       TMEM allocator + tcgen05.mma issuer (the whole warp runs the
+//                issue loop; elect.sync picks the issuing lane)
+//   warp 2       TMA producer for q (one 32 KB load per sequence segment);
+//                with an FP8 cache also the segment publisher
+//   warp 3       bf16 cache: segment publisher; FP8 cache: q converter (q to
+//                its exact E4M3 pair, a segment ahead)
 //   warps 4-7    softmax warpgroup 0: heads 0-31  } thread = one token row of S^T,
 //   warps 8-11   softmax warpgroup 1: heads 32-63 } then one head-dim row of O^T
 //
@@ -73,79 +78,115 @@ __device__ int g_mfa_cnt[2 * kGtCtas];  // per (kernel, CTA) call counter
 
 namespace {
 
-constexpr int kWG = 2;  // softmax warpgroups
-constexpr int kWGHeads = kHeads / kWG;
+// Softmax warpgroups. bf16 cache: two, heads 0-31 | 32-63 (HBM-bound; 168
+// registers a thread). FP8 cache: four of 16 heads each: its tile rate is bound
+// by the softmax chain, which shorter rows and more warps in flight shorten.
+template <bool kFp8>
+struct Geo {
+  static constexpr int kWG = kFp8 ? 4 : 2;
+  static constexpr int kWGHeads = kHeads / kWG;
+  static constexpr int kThreads = 128 + 128 * kWG;  // 4 service warps + the softmax warps
+  static constexpr int kQGroupWarps = 1 + 4 * kWG;  // FP8 first-segment q conversion group
+};
 
 // ---------------------------------------------------------------------------
 // shared-memory control block
 // ---------------------------------------------------------------------------
+template <bool kFp8>
 struct __align__(16) DecodeCtrl {
+  static constexpr int kWG = Geo<kFp8>::kWG;
+  static constexpr int kWGHeads = Geo<kFp8>::kWGHeads;
   uint64_t q_full[2], q_empty[2];  // per q buffer (FP8: two, alternating by segment)
   uint64_t slot_full[kSlots], slot_empty[kSlots];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, o_full;
   uint64_t q_conv[2];  // FP8 cache: q buffer converted to its E4M3 pair
-  uint64_t red_full[kWG][2], l_full[kWG];
+  uint64_t red_full[kWG][2], l_pre[kWG], l_full[kWG];
   uint64_t drain;
   long long t0;    // first global tile of this CTA (balanced plan)
   long long ntot;  // total tiles of the batch (balanced plan)
   uint32_t tmem_base;
   int abort_flag;
-  unsigned seg_arrivals;  // bf16 cache: softmax-warp arrivals at segment ends (never wraps)
+  unsigned seg_arrivals;  // softmax-warp arrivals at segment ends (never wraps)
   unsigned q_ready;       // FP8 cache: segments whose q is converted (never wraps)
   float qinv[4];          // FP8 cache: score scale 1/s of segment k at [k & 3]
-  unsigned qmax[16];      // FP8 cache: per-warp max |q| bits of the first segment's group conversion
+  unsigned qmax[Geo<kFp8>::kQGroupWarps];  // FP8: per-warp max |q| bits, first segment's conversion
   int b_start, off_start, tiles;
-  int scan_warp[kDecodeThreads / 32];
-  int lens[kDecodeThreads];  // validated seq_lens when batch <= kDecodeThreads
+  int scan_warp[Geo<kFp8>::kThreads / 32];
+  // balanced plan: lens[0] = b_start, lens[1 + k] = validated length of
+  // sequence b_start + k (k < 8)
+  int lens[9];
   // vector-loaded (float4): keep 16-byte aligned
-  alignas(16) float red[2][kWG][4][kWGHeads];  // per-warp tile maxima
-  alignas(16) float mv[kWG][4][kWGHeads];      // per-warp copy: running max in use
-  alignas(16) float cv[kWG][4][kWGHeads];      // per-warp copy: rescale factors / out scale
-  alignas(16) float lred[kWG][4][kWGHeads];    // per-warp partial row sums (epilogue)
-  alignas(16) float ev[kWG][4][kWGHeads];      // per-warp copy: output scale of a segment
+  // [tile parity][warpgroup][warp][head]: per-warp tile maxima; at a
+  // segment's end the same buffer carries the per-warp row sums
+  alignas(16) float red[2][kWG][4][kWGHeads];
+  // [tile parity][warpgroup][head]: the running maximum in use for the tile's
+  // probabilities (the four warps of a warpgroup store the same values)
+  alignas(16) float mv[2][kWG][kWGHeads];
 };
-static_assert(offsetof(DecodeCtrl, red) % 16 == 0 && offsetof(DecodeCtrl, mv) % 16 == 0 &&
-                  offsetof(DecodeCtrl, cv) % 16 == 0 && offsetof(DecodeCtrl, lred) % 16 == 0,
+static_assert(offsetof(DecodeCtrl<false>, red) % 16 == 0 &&
+                  offsetof(DecodeCtrl<false>, mv) % 16 == 0 &&
+                  offsetof(DecodeCtrl<true>, red) % 16 == 0 &&
+                  offsetof(DecodeCtrl<true>, mv) % 16 == 0,
               "vector-loaded control arrays must be 16-byte aligned");
 
-// Shared memory: q buffer(s) | ring | P | control. bf16: one q buffer, five
-// ring slots (HBM-bound: every slot of bytes in flight counts). FP8: two q
-// buffers, so the next segment's q is loaded and converted a whole segment
-// ahead, and four slots (the FP8 kernel is bound by its per-tile pipeline,
-// not by bytes in flight).
+// Shared memory (1024-byte aligned base): q buffer(s) | ring | P | control.
+// bf16: one q buffer, five 32 KB ring slots (HBM-bound: every slot of bytes in
+// flight counts) and a 32 KB P tile (probabilities as a bf16 pair hi + lo, two
+// 16 KB column blocks). FP8: two q buffers, so the next segment's q is loaded
+// and converted a whole segment ahead, four ring slots and a 16 KB P tile (an
+// E4M3 pair, two 8 KB blocks).
 template <bool kFp8>
 struct SmemLayout {
   static constexpr int kQBufs = kFp8 ? 2 : 1;
   static constexpr int kRing = kFp8 ? 4 : kSlots;
+  static constexpr int kPSize = kFp8 ? kPBytes : 2 * kPBytes;
   static constexpr int kQ = 0;
   static constexpr int kRingOff = kQ + kQBufs * kQBytes;
   static constexpr int kP = kRingOff + kRing * kSlotBytes;
-  static constexpr int kCtrl = kP + kPBytes;
-  static constexpr int kBytes = kCtrl + static_cast<int>(sizeof(DecodeCtrl)) + 1024;
+  static constexpr int kCtrl = kP + kPSize;
+  static constexpr int kBytes = kCtrl + static_cast<int>(sizeof(DecodeCtrl<kFp8>));
 };
 static_assert(SmemLayout<false>::kBytes <= 227 * 1024 && SmemLayout<true>::kBytes <= 227 * 1024,
               "shared memory budget");
-static_assert(SmemLayout<true>::kRing <= kSlots, "ring barriers");
+static_assert(SmemLayout<false>::kRing <= kSlots && SmemLayout<true>::kRing <= kSlots,
+              "ring barriers");
 
-// TMEM column map.
-constexpr uint32_t kColS = 0;      // score buffers: bf16 cols 0-63 | 64-127; FP8 0-63 | 256-319
-constexpr uint32_t kColOlo = 128;  // O^T rows 0..127
-constexpr uint32_t kColOhi = 192;  // O^T rows 128..255
-constexpr uint32_t kColObuf = 256; // column offset of the odd segments' O pair
+// bf16 P tile: the hi block and the lo block are 16 KB apart (the LBO of the
+// N = 128 MN-major operand); which comes first depends on the segment (below).
+constexpr uint32_t kPBlock = kPBytes;
 
-__device__ __forceinline__ uint32_t o_cols(int seg) { return (seg & 1) ? kColObuf : 0u; }
+// TMEM column map (512 columns; lane = MMA row, i.e. token row of S^T or
+// head-dim row of O^T; column = head).
+//   scores: tile g's 64 heads at s_cols(g).
+//   O^T, per head-dim half r, the PV product is one N = 128 MMA per step whose
+//   columns hold the products with P's hi part and with its lo part; the
+//   output is their sum.
+//   FP8: 128 columns per half from 128 + 256 r, [hi | lo], single-buffered:
+//        a segment's output is read out at its end.
+//   bf16: 192 columns per half from 128 + 192 r, [hi of even segments | lo |
+//        hi of odd segments]. Even segments write [hi | lo] (P's hi block
+//        first), odd segments [lo | hi] (lo block first), so the hi columns are
+//        double-buffered by segment while the lo columns are shared: at a
+//        segment's end its lo part is added into its hi columns (before the
+//        next segment's first PV overwrites lo), and its hi columns are read
+//        out while the next segment accumulates into the other hi block.
+constexpr uint32_t kColS = 0;
 
-// First column of O^T rows 128 r .. 128 r + 127 (r: head-dim half) for the
-// segment with ordinal seg. bf16: 64 columns (heads), double-buffered by
-// segment. FP8: 128 columns, the products with P's hi part in the first 64
-// and with its lo part in the next 64 (one N = 128 product per step reads each
-// V step once for both parts); single-buffered, so an FP8 segment's output is
-// read out at its end.
 template <bool kFp8>
-__device__ __forceinline__ uint32_t o_base(int seg, int r) {
-  return kFp8 ? (r ? 384u : 128u) : o_cols(seg) + (r ? kColOhi : kColOlo);
+__device__ __forceinline__ uint32_t o_hi(int seg, int r) {
+  return kFp8 ? (r ? 384u : 128u) : 128u + 192u * r + ((seg & 1) ? 128u : 0u);
 }
+template <bool kFp8>
+__device__ __forceinline__ uint32_t o_lo(int seg, int r) {
+  return kFp8 ? (r ? 448u : 192u) : 192u + 192u * r;
+}
+// first column written by the segment's PV products for head-dim half r
+template <bool kFp8>
+__device__ __forceinline__ uint32_t o_pv(int seg, int r) {
+  return kFp8 ? o_hi<kFp8>(seg, r) : 128u + 192u * r + ((seg & 1) ? 64u : 0u);
+}
+static_assert(128 + 192 * 2 == kTmemCols && 384 + 128 == kTmemCols, "TMEM columns");
 
 // Score buffer of tile g: 64 columns (heads). With an FP8 cache the products
 // with q's hi and lo parts accumulate into the same columns (two N = 64
@@ -195,7 +236,7 @@ struct TileStream {
   // never reloads them through memory (the hot loops hold memory-clobbering
   // waits, after which a pointer read would go back out to the cache hierarchy)
   const int* seq_lens;
-  const int* lens;  // shared copy of the lengths, or nullptr
+  const int* lens;  // shared copy of some lengths ({first sequence, 8 lengths}), or nullptr
   int cap_tokens, num_splits, grid, batch;
   int cta;
   int b, tile, L, nt, remaining, seg_lo, seg_hi, seg_ord;
@@ -206,7 +247,7 @@ struct TileStream {
   __device__ void init(const DecodeParams& prm, const int* lens_, int b_start, int off_start,
                        int tiles, long long t0) {
     seq_lens = prm.seq_lens;
-    lens = lens_;
+    lens = prm.num_splits == 0 ? lens_ : nullptr;
     cap_tokens = prm.cap_tokens;
     num_splits = prm.num_splits;
     grid = prm.grid;
@@ -234,7 +275,10 @@ struct TileStream {
 
   // fixed plan: move to the next non-empty unit owned by this CTA
   __device__ int length(int seq) const {
-    if (lens) return lens[seq];
+    if (lens) {
+      const unsigned k = static_cast<unsigned>(seq - lens[0]);
+      if (k < 8u) return lens[1 + k];
+    }
     int n = __ldg(seq_lens + seq);
     if (n < 0 || n > cap_tokens) {
       record_error(5 /* MFA_ERR_BAD_INDEX */);
@@ -284,7 +328,11 @@ struct TileStream {
       t.cta_last = (remaining == 0);
       if (remaining > 0 && tile == nt) {
         do {
-          ++b;
+          if (++b >= batch) {  // lengths that disagree with the plan: stop, reported
+            record_error(5 /* MFA_ERR_BAD_INDEX */);
+            remaining = 0;
+            return true;
+          }
           L = length(b);
           nt = tiles_of(L);
         } while (nt == 0);
@@ -395,46 +443,21 @@ __device__ __forceinline__ bool wait_count(const unsigned* ctr, unsigned target,
   }
 }
 
-// the four ready words of a sequence (32 bytes, 16-byte aligned)
-__device__ __forceinline__ void st_ready4(unsigned long long* dst, unsigned long long v) {
-  asm volatile(
-      "st.volatile.global.v2.b64 [%0], {%1, %1};\n\t"
-      "st.volatile.global.v2.b64 [%0+16], {%1, %1};" ::"l"(dst),
-      "l"(v)
-      : "memory");
-}
-
-// Publishes the end of a segment to the combine kernel (one thread). For a
-// split sequence the call counts as one of `arrivals` x (segments) arrivals;
-// the last one (after whose arrival every partial is in memory: each arriver
-// made its partial visible first) sets the ready words to "merge". A sequence
-// that one segment covers is marked "nothing to merge".
-__device__ __forceinline__ void publish_segment(const DecodeParams& p, const TileInfo& t,
-                                                long long ntot, unsigned arrivals) {
-  unsigned long long word = kReadyNone;
-  if (t.slot >= 0) {
-    // one acquire-release increment: its release half orders this segment's
-    // partial (whose stores this thread has acquired) before the arrival, its
-    // acquire half the other arrivers' partials before what follows; wraps
-    // to 0 on the last arrival
-    const unsigned n = arrivals * static_cast<unsigned>(segments_of(p, t, ntot));
-    unsigned old;
-    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;"
-                 : "=r"(old)
-                 : "l"(p.ws_arrive + t.b), "r"(n - 1)
-                 : "memory");
-    if (old != n - 1) return;
-    word = kReadyMerge | (static_cast<unsigned long long>(t.gtile - t.tile) << 2) |
-           (static_cast<unsigned long long>(ntot) << 32);
-  }
-  // release: everything this thread has observed before the ready words
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-  st_ready4(p.ws_ready + 4 * static_cast<int64_t>(t.b), word);
+// Publishes a split segment's partial to the combine kernel (one thread, once
+// the softmax warps' stores of it are ordered before this thread: their
+// release arrivals on the shared counter, acquired by the caller). The release
+// store makes those stores visible device-wide with the slot's flag. A segment
+// that covers its whole sequence wrote the output itself: nothing to publish.
+__device__ __forceinline__ void publish_segment(const DecodeParams& p, const TileInfo& t) {
+  if (t.slot < 0) return;
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.ws_flag + t.slot), "r"(1u)
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------
 // Block-wide plan: total tiles, this CTA's tile range and its first sequence.
 // ---------------------------------------------------------------------------
+template <int kThreads>
 __device__ int block_inclusive_scan(int v, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -446,7 +469,7 @@ __device__ int block_inclusive_scan(int v, int* warp_sums, int* total) {
   __syncthreads();
   int add = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < kDecodeThreads / 32; ++w) {
+  for (int w = 0; w < kThreads / 32; ++w) {
     if (w < warp) add += warp_sums[w];
     tot += warp_sums[w];
   }
@@ -455,71 +478,93 @@ __device__ int block_inclusive_scan(int v, int* warp_sums, int* total) {
   return v + add;
 }
 
-// Reads and validates the lengths once; when the batch fits (B <= threads)
-// they stay in shared memory for every role.
-__device__ void load_lengths(const DecodeParams& p, DecodeCtrl& c) {
-  if (p.batch <= kDecodeThreads && threadIdx.x < p.batch) c.lens[threadIdx.x] = valid_len(p, threadIdx.x);
-}
-
-__device__ void balanced_plan(const DecodeParams& p, DecodeCtrl& c, const int* lens) {
+// Every CTA computes the whole plan (an exclusive scan of the sequences' tile
+// counts); CTA c also stores the plan words of sequences b = c (mod grid) for
+// the combine kernel.
+template <bool kFp8>
+__device__ void balanced_plan(const DecodeParams& p, DecodeCtrl<kFp8>& c) {
+  constexpr int kThreads = Geo<kFp8>::kThreads;
   const int tid = threadIdx.x;
+  const long long G = p.grid;
   long long total = 0;
   long long t0 = 0;
-  bool located = false;
-  if (lens) {
+  if (p.batch <= kThreads) {
     // single pass: the whole batch is one chunk
-    const int n = tid < p.batch ? tiles_of(lens[tid]) : 0;
+    const int n = tid < p.batch ? tiles_of(valid_len(p, tid)) : 0;
     int chunk;
-    const int incl = block_inclusive_scan(n, c.scan_warp, &chunk);
+    const int incl = block_inclusive_scan<kThreads>(n, c.scan_warp, &chunk);
     total = chunk;
-    const long long G = p.grid;
     t0 = (static_cast<long long>(blockIdx.x) * total) / G;
     const long long excl = incl - n;
     if (tid < p.batch && n > 0 && excl <= t0 && t0 < excl + n) {
       c.b_start = tid;
       c.off_start = static_cast<int>(t0 - excl);
     }
-    located = true;
+    if (tid < p.batch && tid % p.grid == static_cast<int>(blockIdx.x))
+      p.ws_plan[tid] = static_cast<unsigned long long>(excl) |
+                       (static_cast<unsigned long long>(total) << 32);
   } else {
-    for (int base = 0; base < p.batch; base += kDecodeThreads) {
+    for (int base = 0; base < p.batch; base += kThreads) {
       const int b = base + tid;
       const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
       int chunk;
-      block_inclusive_scan(n, c.scan_warp, &chunk);
+      block_inclusive_scan<kThreads>(n, c.scan_warp, &chunk);
       total += chunk;
     }
-    t0 = (static_cast<long long>(blockIdx.x) * total) / p.grid;
-  }
-  const long long t1 = (static_cast<long long>(blockIdx.x + 1) * total) / p.grid;
-  if (tid == 0) {
-    c.tiles = static_cast<int>(t1 - t0);
-    c.t0 = t0;
-    c.ntot = total;
-  }
-  if (!located) {
+    t0 = (static_cast<long long>(blockIdx.x) * total) / G;
     long long run = 0;
-    for (int base = 0; base < p.batch && run <= t0; base += kDecodeThreads) {
+    for (int base = 0; base < p.batch; base += kThreads) {
       const int b = base + tid;
       const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
       int chunk;
-      const int incl = block_inclusive_scan(n, c.scan_warp, &chunk);
+      const int incl = block_inclusive_scan<kThreads>(n, c.scan_warp, &chunk);
       const long long excl = run + incl - n;
       if (b < p.batch && n > 0 && excl <= t0 && t0 < excl + n) {
         c.b_start = b;
         c.off_start = static_cast<int>(t0 - excl);
       }
+      if (b < p.batch && b % p.grid == static_cast<int>(blockIdx.x))
+        p.ws_plan[b] = static_cast<unsigned long long>(excl) |
+                       (static_cast<unsigned long long>(total) << 32);
       run += chunk;
     }
   }
+  const long long t1 = (static_cast<long long>(blockIdx.x + 1) * total) / G;
+  if (tid == 0) {
+    c.tiles = static_cast<int>(t1 - t0);
+    c.t0 = t0;
+    c.ntot = total;
+  }
   __syncthreads();
+}
+
+// Fixed split: the next call's L2 warm-up hint, where this CTA's first unit
+// begins (out of line: it runs once, by one thread).
+__device__ __noinline__ void fixed_plan_hint(const int* seq_lens, int cap_tokens, int num_splits,
+                                             int* hint, bool has_units) {
+  int hb = -1, ht = 0;
+  if (has_units) {
+    const int b = static_cast<int>(blockIdx.x) / num_splits;
+    const int j = static_cast<int>(blockIdx.x) % num_splits;
+    const int L = __ldg(seq_lens + b);
+    const int nt = (L < 0 || L > cap_tokens) ? 0 : tiles_of(L);  // (reported by the plan)
+    const int lo = static_cast<int>((static_cast<long long>(j) * nt) / num_splits);
+    const int hi = static_cast<int>((static_cast<long long>(j + 1) * nt) / num_splits);
+    if (hi > lo) {
+      hb = b;
+      ht = lo;
+    }
+  }
+  hint[2 * blockIdx.x] = hb;
+  hint[2 * blockIdx.x + 1] = ht;
 }
 
 // ---------------------------------------------------------------------------
 // warp-level "reduce-scatter": on entry each lane has 32 per-head values of its
 // own row; on exit lane l holds the reduction over all 32 lanes for head l.
 // ---------------------------------------------------------------------------
-template <bool kMax, int N, int MASK>
-__device__ __forceinline__ void rs_step(float (&v)[kWGHeads], int lane) {
+template <bool kMax, int N, int MASK, int NV>
+__device__ __forceinline__ void rs_step(float (&v)[NV], int lane) {
   const bool upper = (lane & MASK) != 0;
 #pragma unroll
   for (int i = 0; i < N / 2; ++i) {
@@ -530,14 +575,26 @@ __device__ __forceinline__ void rs_step(float (&v)[kWGHeads], int lane) {
   }
 }
 
-template <bool kMax>
-__device__ __forceinline__ float reduce_scatter32(float (&v)[kWGHeads], int lane) {
-  rs_step<kMax, 32, 16>(v, lane);
-  rs_step<kMax, 16, 8>(v, lane);
-  rs_step<kMax, 8, 4>(v, lane);
-  rs_step<kMax, 4, 2>(v, lane);
-  rs_step<kMax, 2, 1>(v, lane);
-  return v[0];
+// NV = 32: lane l returns the reduction of value l over the 32 lanes. NV = 16:
+// lanes 2j and 2j + 1 both return the reduction of value j.
+template <bool kMax, int NV>
+__device__ __forceinline__ float reduce_scatter(float (&v)[NV], int lane) {
+  if constexpr (NV == 32) {
+    rs_step<kMax, 32, 16>(v, lane);
+    rs_step<kMax, 16, 8>(v, lane);
+    rs_step<kMax, 8, 4>(v, lane);
+    rs_step<kMax, 4, 2>(v, lane);
+    rs_step<kMax, 2, 1>(v, lane);
+    return v[0];
+  } else {
+    static_assert(NV == 16, "16 or 32 values per lane");
+    rs_step<kMax, 16, 16>(v, lane);
+    rs_step<kMax, 8, 8>(v, lane);
+    rs_step<kMax, 4, 4>(v, lane);
+    rs_step<kMax, 2, 2>(v, lane);
+    const float o = __shfl_xor_sync(0xffffffffu, v[0], 1);
+    return kMax ? fmaxf(v[0], o) : v[0] + o;
+  }
 }
 
 // Ring items per tensor and tile: bf16 K or V tiles take two 32 KB slots (head
@@ -700,7 +757,7 @@ __device__ __forceinline__ float q_to_e4m3(uint32_t base, int lane) {
 // (named barrier 1) of the whole group, the first of which also orders every
 // read of q before the in-place writes. The softmax warps only arrive at the
 // second; warp 3 waits there, then publishes.
-constexpr int kQGroupWarps = 1 + 4 * kWG;
+constexpr int kQGroupWarps = Geo<true>::kQGroupWarps;
 constexpr int kQGroupThreads = 32 * kQGroupWarps;
 static_assert(kQGroupThreads * kQUnitsPerThread >= kQUnits, "group covers q in one round");
 __device__ __forceinline__ float q_to_e4m3_group(uint32_t base, int gtid, bool work, bool publisher,
@@ -734,27 +791,25 @@ constexpr int kCombineHeads = 16;  // heads per CTA
 constexpr int kCombineDims = 16;   // head-dim elements per thread (kDim / 16 threads per head)
 constexpr int kCombineBatch = 4;   // partials loaded per round trip
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* w) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* w) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(w) : "memory");
   return v;
 }
 
-// Waits (bounded) until *w is non-zero; returns it, or 0 after the wait limit.
-// Polls with acquire loads, ordering the caller's reads of the partials after
-// the word.
-__device__ unsigned long long wait_ready(const unsigned long long* w) {
-  unsigned long long v = ld_acquire_u64(w);
-  if (v == 0) {
-    const uint64_t t0 = global_timer_ns();
-    while ((v = ld_acquire_u64(w)) == 0) {
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        record_error(6 /* MFA_ERR_TIMEOUT */);
-        return 0;
-      }
+// Waits (bounded by limit_ns) until the flag is set; false after the limit
+// (MFA_ERR_TIMEOUT recorded). Polls with acquire loads, ordering the caller's
+// reads of the partial after the flag.
+__device__ bool wait_flag(const unsigned* f, unsigned long long limit_ns) {
+  if (ld_acquire_u32(f) != 0) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_u32(f) == 0) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      record_error(6 /* MFA_ERR_TIMEOUT */);
+      return false;
     }
   }
-  return v;
+  return true;
 }
 
 // 16 consecutive output elements of (b, h) from d0 (16-byte vector stores
@@ -847,15 +902,17 @@ __device__ __forceinline__ void merge_head_part(const DecodeParams& p, int b, co
   if (p.lse_out && d0 == 0) p.lse_out[b * p.lse_sb + h] = m + lg2_approx(l) * kLn2;
 }
 
-// The split list of sequence b from its ready word (state kReadyMerge).
-__device__ __forceinline__ SplitList split_list_of(const DecodeParams& p, int b, int nt,
-                                                   unsigned long long word) {
+// The split list of sequence b (nt > 0 tiles): from its plan word (balanced
+// plan), or from the fixed split.
+__device__ __forceinline__ SplitList split_list_of(const DecodeParams& p, int b, int nt) {
   SplitList sl;
-  if (p.num_splits == 0)
-    sl.init_balanced(static_cast<long long>((word & 0xffffffffull) >> 2), nt,
+  if (p.num_splits == 0) {
+    const unsigned long long word = __ldcg(p.ws_plan + b);
+    sl.init_balanced(static_cast<long long>(word & 0xffffffffull), nt,
                      static_cast<long long>(word >> 32), p.grid);
-  else
+  } else {
     sl.init_fixed(b, nt, p.num_splits);
+  }
   return sl;
 }
 
@@ -863,44 +920,63 @@ __device__ __forceinline__ SplitList split_list_of(const DecodeParams& p, int b,
 
 // A finished segment's output, read by one softmax warp: its 32 heads
 // (columns from tcol) for head-dim rows `row` and 128 + `row` (O^T rows in
-// TMEM lanes), scaled per head by ev; the output (slot < 0) or the partial of a
+// TMEM lanes), scaled per head by the output scale that lane `head` holds in
+// ev; the output (slot < 0) or the partial of a
 // split sequence (layout [slot][head][d]: a warp writes 128 contiguous bytes
-// per head). Out of line: it runs once per segment, and its code inlined in
-// the softmax loop (two or three copies) measurably slowed that loop.
+// per head). The accumulator of half r is the hi columns hi_r plus, when
+// add_lo, the lo columns lo_r (a bf16 segment whose lo part was already added
+// into its hi columns passes add_lo = false). Out of line: it runs once per
+// segment, and its code inlined in the softmax loop (two or three copies)
+// measurably slowed that loop.
+template <int W>
+__device__ __forceinline__ void tmem_ldw(uint32_t taddr, uint32_t (&r)[W]) {
+  if constexpr (W == 32)
+    tmem_ld32(taddr, r);
+  else
+    tmem_ld16(taddr, r);
+}
+
 template <bool kFp8>
 __device__ __noinline__ void segment_out(float* ws_o, void* out, int out_f32, int64_t out_sb,
                                          int64_t out_sh, int slot, int b, uint32_t tcol,
-                                         uint32_t o_lo, uint32_t o_hi, int row, int hbase,
-                                         const float* ev) {
+                                         uint32_t hi0, uint32_t hi1, uint32_t lo0, uint32_t lo1,
+                                         bool add_lo, int row, int hbase, float ev, int gqa) {
+  constexpr int W = Geo<kFp8>::kWGHeads;  // this warp's heads (columns)
 #pragma unroll 1
   for (int half = 0; half < 2; ++half) {
-    const int d = half * 128 + row;
-    uint32_t r[32];
-    const uint32_t col = tcol + (half ? o_hi : o_lo);
-    tmem_ld32(col, r);
-    if (kFp8) {  // O = (V P_hi) + (V P_lo)
-      uint32_t r2[32];
-      tmem_ld32(col + 64, r2);
+    // grouped-query mode: this warpgroup's heads form one group, whose output
+    // is O^T's head-dim half of that group (out rows of 128 dims)
+    if (gqa && half != (hbase >> 5)) continue;
+    const int d = gqa ? row : half * 128 + row;
+    uint32_t r[W];
+    tmem_ldw<W>(tcol + (half ? hi1 : hi0), r);
+    if (add_lo) {  // O = (V P_hi) + (V P_lo)
+      uint32_t r2[W];
+      tmem_ldw<W>(tcol + (half ? lo1 : lo0), r2);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
+      for (int j = 0; j < W; ++j)
         r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
     } else {
       tmem_wait_ld();
     }
+    // per head j: the output scale held by lane j
+#pragma unroll
+    for (int j = 0; j < W; ++j)
+      r[j] = __float_as_uint(__uint_as_float(r[j]) * __shfl_sync(0xffffffffu, ev, j));
     if (slot >= 0) {
       float* dst = ws_o + static_cast<int64_t>(slot) * kPartialFloats +
                    static_cast<int64_t>(hbase) * kDim + d;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[j * kDim] = __uint_as_float(r[j]) * ev[j];
+      for (int j = 0; j < W; ++j) dst[j * kDim] = __uint_as_float(r[j]);
     } else if (out_f32) {
       float* dst = static_cast<float*>(out) + b * out_sb + hbase * out_sh + d;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[j * out_sh] = __uint_as_float(r[j]) * ev[j];
+      for (int j = 0; j < W; ++j) dst[j * out_sh] = __uint_as_float(r[j]);
     } else {
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + b * out_sb + hbase * out_sh + d;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[j * out_sh] = __float2bfloat16_rn(__uint_as_float(r[j]) * ev[j]);
+      for (int j = 0; j < W; ++j) dst[j * out_sh] = __float2bfloat16_rn(__uint_as_float(r[j]));
     }
   }
 }
@@ -909,23 +985,30 @@ __device__ __noinline__ void segment_out(float* ws_o, void* out, int out_f32, in
 // the attention kernel
 // ===========================================================================
 template <bool kPaged, bool kFp8>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
+__global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     mfa_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte alignment (the 128-byte swizzle atoms); checked below
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   using L = SmemLayout<kFp8>;
   constexpr uint32_t kS = L::kRing;  // ring slots
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sRing = smem + L::kRingOff;
   uint8_t* sP = smem + L::kP;
-  DecodeCtrl& c = *reinterpret_cast<DecodeCtrl*>(smem + L::kCtrl);
+  constexpr int kWG = Geo<kFp8>::kWG;
+  constexpr int kWGHeads = Geo<kFp8>::kWGHeads;
+  constexpr int kThreads = Geo<kFp8>::kThreads;
+  DecodeCtrl<kFp8>& c = *reinterpret_cast<DecodeCtrl<kFp8>*>(smem + L::kCtrl);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  if (smem_u32(smem_raw) & 1023u) {  // never expected: report, do nothing
+    if (tid == 0) record_error(2 /* MFA_ERR_UNSUPPORTED */);
+    return;
+  }
 
   if (tid == 0) MFA_TR(9, 0);
 #ifdef MFA_TRACE
@@ -950,6 +1033,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     for (int w = 0; w < kWG; ++w) {
       mbar_init(&c.red_full[w][0], 4);
       mbar_init(&c.red_full[w][1], 4);
+      mbar_init(&c.l_pre[w], 4);
       mbar_init(&c.l_full[w], 4);
     }
     mbar_init(&c.p_full, 4 * kWG);
@@ -966,6 +1050,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     tmem_alloc(&c.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  if (!kFp8 && p.gqa) {
+    // Grouped-query mode: group g's 32 heads hold their q (128 dims) in head
+    // dims 128 g .. 128 g + 127 of the 256-wide operand rows and zeros in the
+    // other half, so the score product over 256 dims is the group's own 128-dim
+    // product (q region r = dims 64 r .. 64 r + 63, 128-byte rows). The zero
+    // rows are written once here; q loads never touch them.
+    for (int i = tid; i < 1024; i += kThreads) {
+      const int r = i >> 8, j = i & 255;
+      const int row = (r < 2 ? 32 : 0) + (j >> 3);
+      st_shared_v4(smem_u32(sQ) + r * 8192 + row * 128 + (j & 7) * 16, 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -977,7 +1074,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   // prefetch changes no result: the first K/V tiles this CTA took in the
   // previous call on this workspace (a decode loop's plan barely moves from
   // step to step) are fetched while HBM idles under the previous kernel's tail.
-  if (!kPaged && p.num_splits == 0 && warp == 0 && lane == 0) {
+  if (!kPaged && warp == 0 && lane == 0) {
     const int hb = *reinterpret_cast<volatile const int*>(p.ws_hint + 2 * blockIdx.x);
     const int ht = *reinterpret_cast<volatile const int*>(p.ws_hint + 2 * blockIdx.x + 1);
     if (hb >= 0 && hb < p.batch && ht >= 0 && ht < (p.cap_tokens + kTile - 1) / kTile) {
@@ -991,10 +1088,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   // ---- plan (reads seq_lens: after the previous kernel has completed) -----
   griddep_wait();
-  // The combine kernel may start from here on: it waits for each sequence's
-  // partials on the synchronisation words, which the previous call (complete
-  // now) left at zero.
-  griddep_launch_dependents();
 #ifdef MFA_TRACE
   const int gt_call = blockIdx.x < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[blockIdx.x]) : -1;
   if (tid == 0) {
@@ -1003,23 +1096,40 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       g_mfa_gt[((gt_call * 2) * kGtCtas + blockIdx.x) * 3] = gt_start;
   }
 #endif
-  const int* lens_s = p.batch <= kDecodeThreads ? c.lens : nullptr;
-  load_lengths(p, c);
-  __syncthreads();
+  // balanced plan: the tile streams find the lengths of this CTA's first eight
+  // sequences in shared memory (others in global memory)
+  const int* lens_s = c.lens;
   if (p.num_splits == 0) {
-    balanced_plan(p, c, lens_s);  // ends with __syncthreads
+    balanced_plan(p, c);  // ends with __syncthreads
     if (tid == 0) {  // the next call's L2 warm-up hint
       p.ws_hint[2 * blockIdx.x] = c.tiles > 0 ? c.b_start : -1;
       p.ws_hint[2 * blockIdx.x + 1] = c.off_start;
     }
+    if (tid < 8) c.lens[1 + tid] = c.b_start + tid < p.batch ? valid_len(p, c.b_start + tid) : 0;
+    if (tid == 8) c.lens[0] = c.b_start;
   } else if (tid == 0) {
     c.tiles = static_cast<int>(blockIdx.x) < p.batch * p.num_splits ? -1 : 0;
     c.t0 = 0;
     c.ntot = 0;
+    fixed_plan_hint(p.seq_lens, p.cap_tokens, p.num_splits, p.ws_hint, c.tiles != 0);
   }
+  // This CTA owns the partial slots it may fill (balanced plan: 2c and 2c + 1;
+  // fixed split: units c, c + grid, ...): their flags start the call at zero.
+  if (p.num_splits == 0) {
+    if (tid < 2) p.ws_flag[2 * blockIdx.x + tid] = 0u;
+  } else {
+    const long long units = static_cast<long long>(p.batch) * p.num_splits;
+    for (long long u = blockIdx.x + static_cast<long long>(tid) * p.grid; u < units;
+         u += static_cast<long long>(kThreads) * p.grid)
+      p.ws_flag[u] = 0u;
+  }
+  // The plan words and cleared flags are in place before the combine kernel
+  // may start: it starts once every CTA of this grid has passed this trigger.
+  __threadfence();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_launch_dependents();
 
   volatile int* abort_flag = &c.abort_flag;
   const uint32_t tmem = c.tmem_base;
@@ -1152,7 +1262,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // products of E4M3 operands straight from the ring (K, V), with q and P
     // each given as an exact E4M3 pair hi + lo (two products per step).
     constexpr uint32_t idesc_qk = idesc_f16(128, 64, kFp8 ? 0 : 1, 0, 0);
-    constexpr uint32_t idesc_pv = idesc_f16(128, kFp8 ? 128 : 64, kFp8 ? 0 : 1, 1, 1);
+    // PV: N = 128, the products with P's hi and lo parts side by side
+    constexpr uint32_t idesc_pv = idesc_f16(128, 128, kFp8 ? 0 : 1, 1, 1);
     constexpr uint32_t kIPT = kItemsPerTensor<kFp8>;
     const uint32_t q_base = smem_u32(sQ);
     const uint32_t ring_base = smem_u32(sRing);
@@ -1187,12 +1298,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         for (int kk = 0; kk < kTile / 32; ++kk)
 #pragma unroll
           for (int r = 0; r < 2; ++r)
-            mma_f8_ss_warp(tmem + o_base<kFp8>(t.seg, r),
+            mma_f8_ss_warp(tmem + o_pv<kFp8>(t.seg, r),
                            sw128_desc(v + r * (kSlotBytes / 2) + kk * 4096, kSlotBytes / 2, 1024),
                            sw64_desc(p_base + kk * 2048, kPBytes / 2, 512), idesc_pv,
                            (t.seg_first && kk == 0) ? 0u : 1u);
         mma_commit_warp(&c.slot_empty[lo % kS]);
       } else {
+        // V: two slots (head dims 0-127 | 128-255), each 128 token rows of
+        // 64-dim chunks (MN-major A); P: 128 token rows of the hi and the lo
+        // block (128 B each), 16 KB apart (one N = 128 MN-major B)
         const uint32_t hi = lo + 1;
         const uint32_t v_lo = ring_base + (lo % kS) * kSlotBytes;
         const uint32_t v_hi = ring_base + (hi % kS) * kSlotBytes;
@@ -1200,13 +1314,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         // them alternately, so consecutive products do not wait on each other
 #pragma unroll
         for (int s = 0; s < kTile / 16; ++s) {
-          mma_f16_ss_warp(tmem + o_base<kFp8>(t.seg, 0),
+          mma_f16_ss_warp(tmem + o_pv<kFp8>(t.seg, 0),
                           sw128_desc(v_lo + s * 2048, kSlotBytes / 2, 1024),
-                          sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                          sw128_desc(p_base + s * 2048, kPBlock, 1024), idesc_pv,
                           (t.seg_first && s == 0) ? 0u : 1u);
-          mma_f16_ss_warp(tmem + o_base<kFp8>(t.seg, 1),
+          mma_f16_ss_warp(tmem + o_pv<kFp8>(t.seg, 1),
                           sw128_desc(v_hi + s * 2048, kSlotBytes / 2, 1024),
-                          sw128_desc(p_base + s * 2048, 8192, 1024), idesc_pv,
+                          sw128_desc(p_base + s * 2048, kPBlock, 1024), idesc_pv,
                           (t.seg_first && s == 0) ? 0u : 1u);
         }
         mma_commit_warp(&c.slot_empty[lo % kS]);
@@ -1300,33 +1414,47 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const uint32_t b = kFp8 ? (k & 1u) : 0u;
         if (!(ok = mbar_wait_warp(&c.q_empty[b], (kFp8 ? par(k >> 1) : par(k)) ^ 1u, abort_flag))) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&c.q_full[b], kQBytes);
-          for (int r = 0; r < 4; ++r)
-            tma_load_3d(sQ + b * kQBytes + r * 8192, &tm_q, &c.q_full[b], r * 64, 0, t.b, policy);
+          if (!kFp8 && p.gqa) {
+            // boxes of 64 dims x 32 heads: group g's dims half r into q region
+            // 2 g + r, rows 32 g .. 32 g + 31
+            mbar_arrive_expect_tx(&c.q_full[b], kQBytes / 2);
+            for (int r = 0; r < 4; ++r)
+              tma_load_3d(sQ + b * kQBytes + r * 8192 + (r >> 1) * 4096, &tm_q, &c.q_full[b],
+                          (r & 1) * 64, (r >> 1) * 32, t.b, policy);
+          } else {
+            mbar_arrive_expect_tx(&c.q_full[b], kQBytes);
+            for (int r = 0; r < 4; ++r)
+              tma_load_3d(sQ + b * kQBytes + r * 8192, &tm_q, &c.q_full[b], r * 64, 0, t.b, policy);
+          }
         }
         // pull the next segment's q rows into L2 while this segment runs
         while (more_ahead && (ta.b == t.b || !ta.seg_first)) more_ahead = ahead.next(ta);
-        if (more_ahead && lane == 0)
-          for (int r = 0; r < 4; ++r) tma_prefetch_3d(&tm_q, r * 64, 0, ta.b);
+        if (more_ahead && lane == 0) {
+          if (!kFp8 && p.gqa) {
+            for (int r = 0; r < 4; ++r) tma_prefetch_3d(&tm_q, (r & 1) * 64, (r >> 1) * 32, ta.b);
+          } else {
+            for (int r = 0; r < 4; ++r) tma_prefetch_3d(&tm_q, r * 64, 0, ta.b);
+          }
+        }
         __syncwarp();
         ++k;
-        if (kFp8 && have_last) {
+        if (kFp8 && have_last && last.slot >= 0) {
           if (!(ok = __all_sync(0xffffffffu,
                                 wait_count(&c.seg_arrivals, 4u * kWG * (k - 1), abort_flag))))
             break;
-          if (lane == 0) publish_segment(p, last, c.ntot, 1u);
+          if (lane == 0) publish_segment(p, last);
           __syncwarp();
-          have_last = false;
         }
+        have_last = false;
       }
       if (kFp8 && t.seg_last) {
         last = t;
         have_last = true;
       }
     }
-    if (kFp8 && ok && have_last &&
+    if (kFp8 && ok && have_last && last.slot >= 0 &&
         __all_sync(0xffffffffu, wait_count(&c.seg_arrivals, 4u * kWG * k, abort_flag))) {
-      if (lane == 0) publish_segment(p, last, c.ntot, 1u);
+      if (lane == 0) publish_segment(p, last);
       __syncwarp();
     }
   } else if (warp == 3) {
@@ -1372,17 +1500,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       while (ns.next(t)) {
         if (!t.seg_last) continue;
         ++k;
+        if (t.slot < 0) continue;  // the output itself: nothing to publish
         if (!__all_sync(0xffffffffu, wait_count(&c.seg_arrivals, 4u * kWG * k, abort_flag))) break;
-        if (lane == 0) publish_segment(p, t, c.ntot, 1u);
+        if (lane == 0) publish_segment(p, t);
         __syncwarp();
       }
     }
   } else if (warp >= 4) {
     // ======================= softmax + epilogue =============================
-    const int wg = (warp - 4) >> 2;   // heads [32 wg, 32 wg + 32)
+    const int wg = (warp - 4) >> 2;   // heads [kWGHeads wg, kWGHeads (wg + 1))
     const int sub = warp & 3;         // TMEM sub-partition of this warp
     const int row = sub * 32 + lane;  // token row in S^T / head-dim row in O^T
     const int hbase = wg * kWGHeads;
+    // per-head values (running maximum, row sums, output scale) live in lane
+    // hl (16-head warpgroups: lanes l and l + 16 both hold head l)
+    const int hl = lane & (kWGHeads - 1);
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
     TileStream ts;
     ts.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
@@ -1397,14 +1529,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     }
     TileInfo t;
     uint32_t g = 0, nseg = 0;
-    float m_run = -INFINITY;  // running max in use (log2 units), head hbase + lane
+    float m_run = -INFINITY;  // running max in use (log2 units), head hbase + hl
     float l_part[kWGHeads];
 #pragma unroll
     for (int h = 0; h < kWGHeads; ++h) l_part[h] = 0.f;
     const float sl2 = p.score_log2;
-    float* mv = c.mv[wg][sub];
-    float* cv = c.cv[wg][sub];
-    float* ev = c.ev[wg][sub];  // output scale of the pending segment, per head
+    float ev = 0.f;  // output scale of the pending segment, head hbase + hl
 
     // Reads a finished segment's O (its own TMEM pair) and writes this warp's
     // share: the normalised output, or the partial of a split sequence. Then
@@ -1414,10 +1544,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     TileInfo pend;
     bool have_pending = false;
     uint32_t pend_g = 0;  // tile counter of the pending segment's last tile
-    auto write_segment = [&](const TileInfo& pt) {
+    auto write_segment = [&](const TileInfo& pt, bool add_lo) {
       segment_out<kFp8>(p.ws_o, p.out, p.out_f32, p.out_sb, p.out_sh, pt.slot, pt.b,
-                        tmem + lane_addr + hbase, o_base<kFp8>(pt.seg, 0), o_base<kFp8>(pt.seg, 1),
-                        row, hbase, ev);
+                        tmem + lane_addr + hbase, o_hi<kFp8>(pt.seg, 0), o_hi<kFp8>(pt.seg, 1),
+                        o_lo<kFp8>(pt.seg, 0), o_lo<kFp8>(pt.seg, 1), add_lo, row, hbase,
+                        ev, kFp8 ? 0 : p.gqa);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) smem_add_release(&c.seg_arrivals, 1u);
@@ -1441,8 +1572,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // scaled scores (log2 units); the maximum's own term is then exactly 0
       float s[kWGHeads];
       {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + s_cols<kFp8>(g) + hbase, r);
+        uint32_t r[kWGHeads];
+        tmem_ldw<kWGHeads>(tmem + lane_addr + s_cols<kFp8>(g) + hbase, r);
         tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < kWGHeads; ++h) s[h] = __uint_as_float(r[h]) * sl2_seg;
@@ -1477,8 +1608,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (lane == 0) mbar_arrive(&c.red_full[wg][g & 1]);
       if (!mbar_wait_warp(&c.red_full[wg][g & 1], par(g >> 1), abort_flag)) break;
       if (warp == 4 && lane == 0) MFA_TR(5, g);
-      const float tmax = fmaxf(fmaxf(c.red[g & 1][wg][0][lane], c.red[g & 1][wg][1][lane]),
-                               fmaxf(c.red[g & 1][wg][2][lane], c.red[g & 1][wg][3][lane]));
+      const float tmax = fmaxf(fmaxf(c.red[g & 1][wg][0][hl], c.red[g & 1][wg][1][hl]),
+                               fmaxf(c.red[g & 1][wg][2][hl], c.red[g & 1][wg][3][hl]));
       // lazy rescaling: move the reference max only when the tile's max
       // exceeds it by more than the threshold (exact: the factor cancels)
       float corr = 1.f;
@@ -1487,16 +1618,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         m_run = tmax;
       }
       const bool rescale = __any_sync(0xffffffffu, corr != 1.f);
-      mv[lane] = m_run;
-      cv[lane] = corr;
+      float* mv = c.mv[g & 1][wg];  // every warp of the warpgroup stores the same values
+      mv[hl] = m_run;
       __syncwarp();
 
       // ---- probabilities, row sums ---------------------------------------
       if (rescale) {  // (rare) the row sums move to the new reference first
 #pragma unroll
-        for (int h = 0; h < kWGHeads; ++h) l_part[h] *= cv[h];
+        for (int h = 0; h < kWGHeads; ++h) l_part[h] *= __shfl_sync(0xffffffffu, corr, h);
       }
+      // packed P: bf16 hi parts in pk, lo parts (p - hi, rounded) in pl; FP8
+      // E4M3 hi bytes in pk[0..7], lo bytes in pk[8..15]
       uint32_t pk[kWGHeads / 2];
+      uint32_t pl[kFp8 ? 1 : kWGHeads / 2];
 #pragma unroll
       for (int h = 0; h < kWGHeads; h += 4) {
         const float4 m4 = *reinterpret_cast<const float4*>(&mv[h]);
@@ -1509,13 +1643,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         l_part[h + 2] += p2;
         l_part[h + 3] += p3;
         if (kFp8) {
-          // E4M3 pairs: hi bytes of heads h..h+3 in pk[h / 4], lo bytes in pk[8 + h / 4]
+          // E4M3 pairs: hi bytes of heads h..h+3 in pk[h / 4], lo bytes in
+          // pk[kWGHeads / 4 + h / 4]
           const uint32_t a = split_e4m3x2(p0, p1), b = split_e4m3x2(p2, p3);
           pk[h / 4] = (a & 0xFFFFu) | (b << 16);
-          pk[8 + h / 4] = (a >> 16) | (b & 0xFFFF0000u);
+          pk[kWGHeads / 4 + h / 4] = (a >> 16) | (b & 0xFFFF0000u);
         } else {
-          pk[h / 2] = pack_bf16x2(p0, p1);
-          pk[h / 2 + 1] = pack_bf16x2(p2, p3);
+          // p = hi + lo to ~16 significant bits: the PV product's error is then
+          // far below that of a single bf16 rounding (2^-9 relative)
+          const uint32_t a = pack_bf16x2(p0, p1), b = pack_bf16x2(p2, p3);
+          pk[h / 2] = a;
+          pk[h / 2 + 1] = b;
+          pl[h / 2] = pack_bf16x2(p0 - __uint_as_float(a << 16), p1 - __uint_as_float(a & 0xFFFF0000u));
+          pl[h / 2 + 1] =
+              pack_bf16x2(p2 - __uint_as_float(b << 16), p3 - __uint_as_float(b & 0xFFFF0000u));
         }
       }
 
@@ -1524,53 +1665,91 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (g >= 1 && !mbar_wait_warp(&c.o_full, par(g - 1), abort_flag)) break;
       tc_fence_after();
       if (rescale && !t.seg_first) {
+        constexpr int kChunks = kWGHeads / 16;  // 16-column chunks of this warp's heads
 #pragma unroll 1
-        for (int q4 = 0; q4 < (kFp8 ? 8 : 4); ++q4) {  // halves x two 16-column chunks (x 2 parts)
+        for (int q4 = 0; q4 < 4 * kChunks; ++q4) {  // (hi, lo) x halves x chunks
           uint32_t r[16];
-          const int cb = (q4 & 1) * 16;
-          const uint32_t a = tmem + lane_addr + o_base<kFp8>(t.seg, (q4 >> 1) & 1) + (q4 >> 2) * 64 +
-                             hbase + cb;
+          const int cb = (q4 % kChunks) * 16, half = (q4 / kChunks) & 1;
+          const uint32_t a =
+              tmem + lane_addr +
+              ((q4 / (2 * kChunks)) ? o_lo<kFp8>(t.seg, half) : o_hi<kFp8>(t.seg, half)) + hbase +
+              cb;
           tmem_ld16(a, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * cv[cb + j]);
+          for (int j = 0; j < 16; ++j)
+            r[j] = __float_as_uint(__uint_as_float(r[j]) * __shfl_sync(0xffffffffu, corr, cb + j));
           tmem_st16(a, r);
+        }
+        tmem_wait_st();
+      }
+      if (!kFp8 && have_pending) {
+        // first tile of a new segment (bf16): the previous segment's last PV
+        // has completed (the wait above); add its lo part into its hi columns
+        // before this tile's PV overwrites the shared lo columns
+        constexpr int kChunks = kWGHeads / 16;
+#pragma unroll 1
+        for (int q4 = 0; q4 < 2 * kChunks; ++q4) {  // halves x 16-column chunks
+          uint32_t a[16], b[16];
+          const int cb = (q4 % kChunks) * 16, half = q4 / kChunks;
+          const uint32_t ha = tmem + lane_addr + o_hi<kFp8>(pend.seg, half) + hbase + cb;
+          tmem_ld16(ha, a);
+          tmem_ld16(tmem + lane_addr + o_lo<kFp8>(pend.seg, half) + hbase + cb, b);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            a[j] = __float_as_uint(__uint_as_float(a[j]) + __uint_as_float(b[j]));
+          tmem_st16(ha, a);
         }
         tmem_wait_st();
       }
       if (kFp8) {
         // P hi | lo: 128 token rows of 64 heads (64 B, 64-byte swizzle); this
-        // warpgroup's 32 heads are 16-byte chunks 2 wg, 2 wg + 1 of the row
+        // warpgroup's heads are the row's 16-byte chunks kC wg .. kC wg + kC - 1
+        constexpr int kC = kWGHeads / 16;
         const uint32_t rowaddr = smem_u32(sP) + row * 64;
         const int sw = (row >> 1) & 3;
 #pragma unroll
         for (int part = 0; part < 2; ++part)
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch)
-            st_shared_v4(rowaddr + part * (kPBytes / 2) + (((2 * wg + ch) ^ sw) << 4),
-                         pk[8 * part + 4 * ch], pk[8 * part + 4 * ch + 1],
-                         pk[8 * part + 4 * ch + 2], pk[8 * part + 4 * ch + 3]);
+          for (int ch = 0; ch < kC; ++ch)
+            st_shared_v4(rowaddr + part * (kPBytes / 2) + (((kC * wg + ch) ^ sw) << 4),
+                         pk[(kWGHeads / 4) * part + 4 * ch], pk[(kWGHeads / 4) * part + 4 * ch + 1],
+                         pk[(kWGHeads / 4) * part + 4 * ch + 2],
+                         pk[(kWGHeads / 4) * part + 4 * ch + 3]);
       } else {
+        // P hi and lo blocks: 128 token rows of 64 heads (128 B, 128-byte
+        // swizzle); this warpgroup's heads are 16-byte chunks kC wg ..
+        // kC wg + kC - 1. Even segments put the hi block first, odd ones the lo
+        // block (the TMEM column map above).
+        constexpr int kC = kWGHeads / 8;
         const uint32_t rowaddr = smem_u32(sP) + row * 128;
+        const uint32_t hi_off = (t.seg & 1) ? kPBlock : 0u;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          st_shared_v4(rowaddr + (((4 * wg + ch) ^ (row & 7)) << 4), pk[4 * ch], pk[4 * ch + 1],
-                       pk[4 * ch + 2], pk[4 * ch + 3]);
+        for (int ch = 0; ch < kC; ++ch) {
+          const uint32_t a = rowaddr + (((kC * wg + ch) ^ (row & 7)) << 4);
+          st_shared_v4(a + hi_off, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          st_shared_v4(a + (kPBlock - hi_off), pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2],
+                       pl[4 * ch + 3]);
+        }
       }
       // rows past the sequence end: zero the V rows so 0 * (stale or NaN) never
-      // reaches the accumulator (warpgroup 0: head dims 0-127, 1: 128-255;
-      // bf16: the item of those dims, two 64-dim regions; FP8: that half of
-      // the tensor's one item)
+      // reaches the accumulator. bf16 (two warpgroups): warpgroup w takes the
+      // item of head dims 128 w .. 128 w + 127 (two 64-dim regions). FP8: the
+      // tensor's one item (two 16 KB halves of 128-byte rows); warpgroup w
+      // takes half w & 1, bytes kRowPart (w >> 1) .. + kRowPart - 1 of each row.
       if (valid < kTile) {
+        constexpr int kRowPart = kFp8 ? 256 / kWG : 128;  // bytes of a 128-byte row
         const uint32_t it = v_item<kFp8>(g, t.cta_last) + (kFp8 ? 0 : wg);
         if (!mbar_wait_warp(&c.slot_full[it % kS], par(it / kS), abort_flag)) break;
         if (!row_ok) {
-          const uint32_t base = smem_u32(sRing) + (it % kS) * kSlotBytes + row * 128 +
-                                (kFp8 ? wg * (kSlotBytes / 2) : 0);
+          const uint32_t base =
+              smem_u32(sRing) + (it % kS) * kSlotBytes + row * 128 +
+              (kFp8 ? (wg & 1) * (kSlotBytes / 2) + (wg >> 1) * kRowPart : 0);
 #pragma unroll
           for (int r = 0; r < (kFp8 ? 1 : 2); ++r)
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
+            for (int ch = 0; ch < kRowPart / 16; ++ch)
               st_shared_v4(base + r * (kSlotBytes / 2) + ch * 16, 0u, 0u, 0u, 0u);
         }
       }
@@ -1587,29 +1766,41 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // segment is read out at its end or after the loop, never here: the
       // condition keeps this copy of the read-out out of the FP8 loop's code.)
       if (!kFp8 && have_pending) {
-        write_segment(pend);
+        write_segment(pend, false);  // its lo part is in its hi columns now
         have_pending = false;
       }
 
       // ---- end of a segment: row sums and log-sum-exp ---------------------
       if (t.seg_last) {
+        // the row sums travel through this tile's maxima buffer, once every
+        // warp of the warpgroup has read its maxima (l_pre); it is next
+        // written two tiles on, after every warp has passed the next tile's
+        // maximum exchange (so after the reads below)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.l_pre[wg]);
+        if (!mbar_wait_warp(&c.l_pre[wg], par(nseg), abort_flag)) break;
+        float* lred = &c.red[g & 1][wg][0][0];
         {
           float v[kWGHeads];
 #pragma unroll
           for (int h = 0; h < kWGHeads; ++h) v[h] = l_part[h];
-          c.lred[wg][sub][lane] = reduce_scatter32<false>(v, lane);
+          const float rs = reduce_scatter<false>(v, lane);
+          if (kWGHeads == 32)
+            lred[sub * kWGHeads + lane] = rs;
+          else if ((lane & 1) == 0)
+            lred[sub * kWGHeads + (lane >> 1)] = rs;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&c.l_full[wg]);
         if (!mbar_wait_warp(&c.l_full[wg], par(nseg), abort_flag)) break;
-        const float l = c.lred[wg][0][lane] + c.lred[wg][1][lane] + c.lred[wg][2][lane] +
-                        c.lred[wg][3][lane];
+        const float l = lred[hl] + lred[kWGHeads + hl] + lred[2 * kWGHeads + hl] +
+                        lred[3 * kWGHeads + hl];
         // the next tile starts a new segment: the row sums restart from zero
 #pragma unroll
         for (int h = 0; h < kWGHeads; ++h) l_part[h] = 0.f;
-        const float lse = (m_run + lg2_approx(l)) * kLn2;  // head hbase + lane
-        ev[lane] = p.out_scale / l;
-        if (sub == 0) {
+        const float lse = (m_run + lg2_approx(l)) * kLn2;  // head hbase + hl
+        ev = p.out_scale / l;
+        if (sub == 0 && lane < kWGHeads) {
           if (t.slot >= 0)
             p.ws_lse[static_cast<int64_t>(t.slot) * kHeads + hbase + lane] = lse;
           else if (p.lse_out)
@@ -1624,7 +1815,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           // single O buffer: read out now, before the next segment's first PV
           if (!mbar_wait_warp(&c.o_full, par(g), abort_flag)) break;
           tc_fence_after();
-          write_segment(pend);
+          write_segment(pend, true);
           have_pending = false;
         }
       }
@@ -1633,7 +1824,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     // the CTA's last segment: after its last PV
     if (have_pending && !*abort_flag && mbar_wait_warp(&c.o_full, par(g - 1), abort_flag)) {
       tc_fence_after();
-      write_segment(pend);
+      write_segment(pend, true);
     }
   }
 
@@ -1659,10 +1850,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 // over the sequence's partials in plan order.
 //
 // The kernel starts while the attention kernel still runs (on SMs it has
-// left) and merges each sequence as soon as its ready word says its partials
-// are written, so merges overlap the attention kernel's last tiles. One CTA
-// waits for the attention grid to complete at its end, so a call is over when
-// this kernel is.
+// left), once every attention CTA has written its plan words and cleared its
+// slot flags. A CTA derives its sequence's partial slots from the plan, waits
+// (bounded) for their flags and merges, so merges overlap the attention
+// kernel's last tiles; a sequence that one segment covers was finished by the
+// attention kernel itself. One CTA waits for the attention grid to complete at
+// its end, so a call is over when this kernel is.
 // ===========================================================================
 __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams p) {
 #ifdef MFA_TRACE
@@ -1677,12 +1870,6 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
   // the lengths are an input of the call: complete before the attention
   // kernel passed its own dependency wait, which precedes this kernel's start
   const int nt = tiles_of(valid_len(p, b));
-
-  __shared__ unsigned long long s_word;
-  unsigned long long* ready = p.ws_ready + 4 * static_cast<int64_t>(b) + q;
-  if (nt > 0 && threadIdx.x == 0) s_word = wait_ready(ready);
-  __syncthreads();
-  const unsigned long long word = nt > 0 ? s_word : 0;
 #ifdef MFA_TRACE
   const int gt_call = cta_lin < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[kGtCtas + cta_lin]) : -1;
   if (threadIdx.x == 0) {
@@ -1702,18 +1889,39 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
   } gt_end{gt_call, cta_lin};
 #endif
 
-  float v[kCombineDims];
+  // grouped-query mode: 128 output dims per head (partials keep their 256-wide
+  // rows, the group's values in the first 128)
+  const bool dims_ok = !p.gqa || d0 < kDim / 2;
   if (nt == 0) {  // empty sequence: zeros, lse = -inf
+    float v[kCombineDims];
 #pragma unroll
     for (int j = 0; j < kCombineDims; ++j) v[j] = 0.f;
-    store_out16(p, b, h, d0, v);
+    if (dims_ok) store_out16(p, b, h, d0, v);
     if (p.lse_out && d0 == 0) p.lse_out[b * p.lse_sb + h] = -INFINITY;
-  } else if ((word & 3) == kReadyMerge) {
-    merge_head_part(p, b, split_list_of(p, b, nt, word), h, d0);
+  } else {
+    const SplitList sl = split_list_of(p, b, nt);
+    // a sequence spans at most grid + 1 CTAs (balanced) or num_splits units
+    const int max_count = p.num_splits == 0 ? p.grid + 1 : p.num_splits;
+    const int nslots = p.num_splits == 0 ? 2 * p.grid : p.batch * p.num_splits;
+    const bool sane = sl.count >= 1 && sl.count <= max_count;
+    if (!sane && threadIdx.x == 0) record_error(5 /* MFA_ERR_BAD_INDEX */);
+    if (sane && sl.nonempty() > 1) {  // split: wait for every partial, then merge
+      __shared__ int s_ok;
+      if (threadIdx.x == 0) s_ok = 1;
+      __syncthreads();
+      for (int i = threadIdx.x; i < sl.count; i += blockDim.x) {
+        const int slot = sl.slot(i);
+        if (slot >= nslots) {
+          record_error(5 /* MFA_ERR_BAD_INDEX */);
+          s_ok = 0;
+        } else if (slot >= 0 && !wait_flag(p.ws_flag + slot, p.wait_ns)) {
+          s_ok = 0;
+        }
+      }
+      __syncthreads();
+      if (s_ok && dims_ok) merge_head_part(p, b, sl, h, d0);
+    }
   }
-  // back to zero for the next call, which sets it only after this kernel
-  // has completed
-  if (nt > 0 && threadIdx.x == 0 && word != 0) *ready = 0;
   // One block waits for the attention grid to complete, so this grid never
   // completes before it: a later kernel that waits for this one (the next
   // call) also waits for the attention kernel. The other blocks leave as soon
@@ -1760,8 +1968,14 @@ static cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk
     if (err != cudaSuccess) return err;
     configured_dev = dev;
   }
-  return launch_pdl(mfa_decode_kernel<kPaged, kFp8>, dim3(p.grid), dim3(kDecodeThreads),
+  return launch_pdl(mfa_decode_kernel<kPaged, kFp8>, dim3(p.grid), dim3(Geo<kFp8>::kThreads),
                     SmemLayout<kFp8>::kBytes, stream, tq, tk, tv, p);
+}
+
+// The combine kernel alone, without programmatic launch (failure self-test).
+cudaError_t launch_combine_only(const DecodeParams& p, cudaStream_t stream) {
+  mfa_combine_kernel<<<dim3(p.batch, kHeads / kCombineHeads), dim3(kDim), 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode(bool paged, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,

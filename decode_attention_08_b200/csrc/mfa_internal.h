@@ -14,14 +14,12 @@ constexpr int kDim = 256;     // head dimension of q and of the shared K / V hea
 constexpr int kTile = 128;    // cached tokens per tile = MMA M of the score product
 
 // Decode-attention kernel geometry (bf16 cache).
-constexpr int kSlots = 5;                  // TMA ring slots
+constexpr int kSlots = 5;                  // TMA ring barriers (the ring uses up to this many slots)
 constexpr int kSlotBytes = 128 * 128 * 2;  // one tensor, 128 tokens x 128 dims, bf16
 constexpr int kQBytes = kHeads * kDim * 2;
-constexpr int kPBytes = kTile * kHeads * 2;
+constexpr int kPBytes = kTile * kHeads * 2;  // one 16-bit P block, or an E4M3 pair
 constexpr int kDecodeThreads = 384;        // 12 warps: 4 service warps + 2 softmax warpgroups
-// S0 | S1 | O_lo | O_hi for even segments | (unused) | O_lo | O_hi for odd
-// segments, 64 columns each: a segment's output is read out while the next
-// segment accumulates into the other pair
+// all of TMEM: score buffers and O^T accumulators (column map in decode_kernel.cu)
 constexpr int kTmemCols = 512;
 
 // One partial (split) result: O [64 heads][256 d] f32, normalised over its range.
@@ -48,21 +46,27 @@ struct DecodeParams {
   int64_t lse_sb;
   float* ws_o;             // [slots][64 heads][256 d] normalised partial outputs
   float* ws_lse;           // [slots][64] their log-sum-exp (natural log)
-  // synchronisation words between the attention and the combine kernel; zero
-  // between calls (each call returns them to zero)
-  unsigned* ws_arrive;     // [B] segment arrivals of a split sequence
-  // [B][4] one word per combine CTA of the sequence: bits 0-1 the state (0
-  // pending, kReadyNone, kReadyMerge), bits 2-31 the sequence's first global
-  // tile, bits 32-63 the batch's total tiles (balanced plan)
-  unsigned long long* ws_ready;
+  // Hand-off between the attention and the combine kernel. Nothing here
+  // carries over from one call to the next, so the workspace needs no
+  // initialisation: every word below is written by the attention kernel
+  // before it lets the combine kernel start (programmatic launch).
+  //   ws_plan [B]: balanced plan, bits 0-31 the sequence's first tile in the
+  //     batch's tile order, bits 32-63 the batch's total tiles.
+  //   ws_flag [slots]: 0 until the slot's partial (and lse) is written in
+  //     this call, then 1; each slot's owner CTA clears it first.
+  unsigned long long* ws_plan;
+  unsigned* ws_flag;
   // [grid][2] where each CTA's tiles began in the previous call on this
   // workspace (first sequence, first tile): a hint for warming L2 before the
   // call's inputs may be read; never trusted for results
   int* ws_hint;
+  // limit of the combine kernel's waits for partials (ns); then it records
+  // MFA_ERR_TIMEOUT and returns
+  unsigned long long wait_ns;
+  // grouped-query mode (bf16 cache): q [B, 64, 128], key/value token rows
+  // [2 groups][128], heads 0-31 in group 0 and 32-63 in group 1, out [B, 64, 128]
+  int gqa;
 };
-
-constexpr unsigned kReadyNone = 1;   // the attention kernel wrote the sequence's output itself
-constexpr unsigned kReadyMerge = 2;  // every partial of the sequence is written
 
 struct QprojParams {
   int batch;

@@ -45,7 +45,9 @@ EXPORTS = ("mfa_decode_attention", "mfa_decode_attention_ex", "mfa_decode_worksp
            "mfa_kv_append", "mfa_kv_append_workspace_size",
            "mfa_output_proj", "mfa_output_proj_workspace_size", "mfa_lse_merge",
            "mfa_read_status", "mfa_error_string", "mfa_version", "mfa_last_cuda_error_string",
-           "mfa_decode_attention_noalloc")
+           "mfa_decode_attention_noalloc", "mfa_selftest_wait_timeout",
+           "mfa_gqa_decode_attention", "mfa_qproj_decode_attention",
+           "mfa_qproj_decode_workspace_size")
 
 
 def lib() -> ctypes.CDLL:
@@ -88,6 +90,17 @@ def lib() -> ctypes.CDLL:
             L.mfa_output_proj_workspace_size.restype = ctypes.c_size_t
             L.mfa_lse_merge.argtypes = [T, T, T, T, P]
             L.mfa_lse_merge.restype = ctypes.c_int
+            L.mfa_gqa_decode_attention.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int,
+                                                   T, P, ctypes.c_size_t, P]
+            L.mfa_gqa_decode_attention.restype = ctypes.c_int
+            L.mfa_qproj_decode_attention.argtypes = [T, T, T, T, T, T, T, T, T, ctypes.c_float,
+                                                     ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                                     ctypes.c_int, T, P, ctypes.c_size_t, P]
+            L.mfa_qproj_decode_attention.restype = ctypes.c_int
+            L.mfa_qproj_decode_workspace_size.argtypes = [ctypes.c_int] * 4
+            L.mfa_qproj_decode_workspace_size.restype = ctypes.c_size_t
+            L.mfa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, P]
+            L.mfa_selftest_wait_timeout.restype = ctypes.c_int
             L.mfa_read_status.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
             L.mfa_read_status.restype = ctypes.c_int
             L.mfa_error_string.argtypes = [ctypes.c_int]
@@ -163,7 +176,7 @@ def decode_attention_ex(q, k_cache, v_cache, page_table, seq_lens, out, softmax_
     """``mfa_decode_attention_ex`` (scales, split control, lse, caller workspace)."""
     need = decode_workspace_size(q.shape[0], num_splits)
     if workspace is None:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)  # needs no zeroing
     rc = lib().mfa_decode_attention_ex(
         describe(q), describe(k_cache), describe(v_cache), describe(page_table),
         describe(seq_lens), describe(out), float(softmax_scale), _kv_code(kv_dtype),
@@ -185,6 +198,49 @@ def decode_attention_noalloc(q, k_cache, v_cache, page_table, seq_lens, out,
         describe(seq_lens), describe(out), float(softmax_scale), _kv_code(kv_dtype),
         float(k_scale), float(v_scale), int(num_splits), describe(lse_out), _stream(stream))
     _check(rc, "mfa_decode_attention_noalloc")
+    return out
+
+
+def gqa_decode_attention(q, k_cache, v_cache, page_table, seq_lens, out,
+                         softmax_scale=1.0 / 128 ** 0.5, num_splits=0, lse_out=None,
+                         workspace: Optional[torch.Tensor] = None, stream=None):
+    """``mfa_gqa_decode_attention``: grouped-query decode attention, q [B, 64, 128],
+    caches [.., 2, 128] bf16 (heads 0-31 use group 0, 32-63 group 1)."""
+    need = decode_workspace_size(q.shape[0], num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib().mfa_gqa_decode_attention(
+        describe(q), describe(k_cache), describe(v_cache), describe(page_table),
+        describe(seq_lens), describe(out), float(softmax_scale), int(num_splits),
+        describe(lse_out), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(rc, "mfa_gqa_decode_attention")
+    return out
+
+
+def qproj_decode_workspace_size(batch: int, dm: int, rank: int, num_splits: int = 0) -> int:
+    return int(lib().mfa_qproj_decode_workspace_size(int(batch), int(dm), int(rank),
+                                                     int(num_splits)))
+
+
+def qproj_decode_attention(x, w_qa, w_qb, q_out, k_cache, v_cache, page_table, seq_lens, out,
+                           softmax_scale=1.0 / 16, kv_dtype="bf16", k_scale=1.0, v_scale=1.0,
+                           num_splits=0, lse_out=None, workspace: Optional[torch.Tensor] = None,
+                           stream=None):
+    """``mfa_qproj_decode_attention``: q_out = (x W_qa) W_qb, then decode attention
+    of q_out (as [B, 64, 256]) over the caches, in one call. A workspace passed
+    in must have had its first 4 KB zeroed before its first use."""
+    if workspace is None:
+        workspace = torch.zeros(qproj_decode_workspace_size(x.shape[0], x.shape[1],
+                                                            w_qa.shape[1], num_splits),
+                                dtype=torch.uint8, device=x.device)
+    rc = lib().mfa_qproj_decode_attention(
+        describe(x), describe(w_qa), describe(w_qb), describe(q_out), describe(k_cache),
+        describe(v_cache), describe(page_table), describe(seq_lens), describe(out),
+        float(softmax_scale), _kv_code(kv_dtype), float(k_scale), float(v_scale),
+        int(num_splits), describe(lse_out), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mfa_qproj_decode_attention")
     return out
 
 
@@ -256,6 +312,13 @@ def lse_merge(o_parts, lse_parts, out, lse_out=None, stream=None):
                              describe(lse_out), _stream(stream))
     _check(rc, "mfa_lse_merge")
     return out
+
+
+def selftest_wait_timeout(wait_ns: int, stream=None) -> None:
+    """``mfa_selftest_wait_timeout``: make one bounded in-kernel wait run out
+    (no fault); read the resulting MFA_ERR_TIMEOUT with ``read_status``."""
+    _check(lib().mfa_selftest_wait_timeout(int(wait_ns), _stream(stream)),
+           "mfa_selftest_wait_timeout")
 
 
 def read_status(stream=None, reset: bool = True) -> int:

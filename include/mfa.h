@@ -110,17 +110,12 @@ int mfa_decode_attention(const mfa_tensor* q, const mfa_tensor* k_cache,
  *                    scores (-inf for empty sequences).
  *  workspace         device memory of at least
  *                    mfa_decode_workspace_size(B, num_splits) bytes, 256-byte
- *                    aligned. Its first bytes hold synchronisation words
- *                    between the call's two kernels, which every call leaves
- *                    at zero. The library clears them itself (one
- *                    cudaMemsetAsync on the call's stream) the first time it
- *                    sees a workspace address and whenever the batch size
- *                    changes, and for every workspace after mfa_read_status
- *                    has reported a non-zero status (a call that gave up a
- *                    wait may leave them set). Between calls the caller must
- *                    not write to the workspace. Calls that overlap on the GPU
- *                    must not share a workspace, and a CUDA graph that
- *                    captured a call needs its workspace to itself.
+ *                    aligned, owned by the caller. It needs no
+ *                    initialisation and its contents between calls do not
+ *                    matter (fresh, reused, or left by another call of any
+ *                    shape): everything the call's second kernel reads from it
+ *                    is written earlier in the same call. Calls that overlap
+ *                    on the GPU must not share a workspace.
  * Splitting never changes which cached rows contribute; the split plan depends
  * only on seq_lens, num_splits and the SM count, never on the cache layout, so a
  * paged and a contiguous cache holding the same rows give bit-identical results.
@@ -131,6 +126,38 @@ int mfa_decode_attention_ex(const mfa_tensor* q, const mfa_tensor* k_cache,
                             int kv_dtype, float k_scale, float v_scale, int num_splits,
                             mfa_tensor* lse_out, void* workspace, size_t workspace_bytes,
                             mfa_stream_t stream);
+
+/*
+ * Grouped-query decode attention (GQA), the comparison shape for MFA (Step-3
+ * summary page, "Key points -> Ablations": MFA beats MLA and GQA in decode
+ * latency; GQA itself is Ainslie et al., in the pages' reference lists). 64
+ * query heads of dimension 128 form 2 groups of 32 consecutive heads; group g
+ * has its own key head and value head of dimension 128, so a cached token costs
+ * 2 x 2 x 128 bf16 = 1024 bytes, exactly MFA's one 256-wide key and value head:
+ *
+ *   out[b,h,:] = softmax_t(softmax_scale * q[b,h,:] . K_b[t,g,:]) V_b[t,g,:],
+ *   g = h / 32, over t < seq_lens[b]   (lse_out as for MFA).
+ *
+ *  q          [B, 64, 128] bf16 (head and batch strides multiples of 8 elements).
+ *  k_cache    contiguous [B, Lmax, 2, 128] or paged [num_pages, page_size, 2, 128],
+ *             bf16; a token's two group rows adjacent (stride 128 elements, d
+ *             stride 1); token and batch/page strides multiples of 16 bytes.
+ *  v_cache    same shape and strides as k_cache.
+ *  page_table, seq_lens, num_splits, lse_out, workspace, stream
+ *             as for mfa_decode_attention_ex (workspace size:
+ *             mfa_decode_workspace_size(B, num_splits)).
+ *  out        [B, 64, 128], MFA_BF16 or MFA_F32, any strides (d stride 1).
+ *  softmax_scale  1/sqrt(128) in the comparison setting.
+ * It runs on the MFA kernels: group g's 128 dims occupy head dims 128 g ..
+ * 128 g + 127 of the 256-wide products (zeros elsewhere), so it issues the same
+ * tensor-core instructions and reads the same bytes per token as MFA.
+ * Returns as mfa_decode_attention_ex; MFA_ERR_UNSUPPORTED for other shapes.
+ */
+int mfa_gqa_decode_attention(const mfa_tensor* q, const mfa_tensor* k_cache,
+                             const mfa_tensor* v_cache, const mfa_tensor* page_table,
+                             const mfa_tensor* seq_lens, mfa_tensor* out, float softmax_scale,
+                             int num_splits, mfa_tensor* lse_out, void* workspace,
+                             size_t workspace_bytes, mfa_stream_t stream);
 
 /* Bytes of workspace mfa_decode_attention_ex needs for `batch` sequences on the
  * current device with the given num_splits. 0 on error. */
@@ -148,13 +175,14 @@ size_t mfa_decode_workspace_size(int batch, int num_splits);
  * on every device that loads the library until the process exits. Requests
  * whose mfa_decode_workspace_size(B, num_splits) exceeds 24 MiB are rejected
  * with MFA_ERR_WORKSPACE (on a 148-SM B200 the default balanced plan needs
- * about 19.5 MiB plus 4 bytes per sequence; with num_splits = s the need is
+ * about 18.6 MiB plus 8 bytes per sequence; with num_splits = s the need is
  * about 64.3 KiB per sequence and split).
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture. Every call on a device uses the same array and nothing
- * in it needs to start at zero, but calls that overlap on the GPU (different
- * streams, or different host threads) race on it: serialise them.
+ * any stream capture. Every call on a device uses the same array, which keeps
+ * the last call's contents; nothing in it needs to start at zero (each call
+ * writes what it reads), but calls that overlap on the GPU (different streams,
+ * or different host threads) race on it: serialise them.
  * Arguments, results and errors are otherwise those of mfa_decode_attention_ex.
  */
 int mfa_decode_attention_noalloc(const mfa_tensor* q, const mfa_tensor* k_cache,
@@ -179,6 +207,33 @@ int mfa_decode_attention_noalloc(const mfa_tensor* q, const mfa_tensor* k_cache,
  */
 int mfa_query_proj(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
                    mfa_tensor* q_out, mfa_stream_t stream);
+
+/*
+ * The query projection followed by decode attention on its result, in one call
+ * (Step-3 page: the queries of every decode token come out of the 2048-wide
+ * bottleneck, then attend over the shared key/value heads):
+ *   q_out = (x * W_qa) * W_qb            as mfa_query_proj_ex, q_out [B, 64 * 256]
+ *   out   = attention(q_out viewed as [B, 64, 256], caches)   as mfa_decode_attention_ex
+ * The projection writes q straight in the layout the attention reads, and the
+ * attention kernel is launched with programmatic dependent launch: its CTAs set
+ * up (barriers, TMEM, an L2 warm-up of their first key/value tiles) on the SMs
+ * the projection's CTAs leave, and read q once the projection has completed.
+ * workspace: mfa_qproj_decode_workspace_size(B, Dm, R, num_splits) bytes,
+ * 256-byte aligned: the projection's workspace (its first 4 KB zero before the
+ * first use, as for mfa_query_proj_ex) followed by the attention's. Arguments
+ * and errors otherwise as the two calls; nothing is launched if either call's
+ * arguments are rejected.
+ */
+int mfa_qproj_decode_attention(const mfa_tensor* x, const mfa_tensor* w_qa,
+                               const mfa_tensor* w_qb, mfa_tensor* q_out,
+                               const mfa_tensor* k_cache, const mfa_tensor* v_cache,
+                               const mfa_tensor* page_table, const mfa_tensor* seq_lens,
+                               mfa_tensor* out, float softmax_scale, int kv_dtype, float k_scale,
+                               float v_scale, int num_splits, mfa_tensor* lse_out,
+                               void* workspace, size_t workspace_bytes, mfa_stream_t stream);
+
+/* Bytes of workspace mfa_qproj_decode_attention needs. 0 on error. */
+size_t mfa_qproj_decode_workspace_size(int batch, int dm, int rank, int num_splits);
 
 /* As mfa_query_proj with a caller workspace of at least
  * mfa_query_proj_workspace_size(B, Dm, R) bytes, 256-byte aligned, that must be
@@ -282,6 +337,21 @@ int mfa_lse_merge(const mfa_tensor* o_parts, const mfa_tensor* lse_parts, mfa_te
  * device's status word: MFA_OK or the first MFA_ERR_BAD_INDEX / MFA_ERR_TIMEOUT
  * a kernel recorded since the last reset. Returns MFA_OK or MFA_ERR_CUDA. */
 int mfa_read_status(mfa_stream_t stream, int reset, int* status_out);
+
+/*
+ * Failure-path self-test (no counterpart on the pages; failure handling is this
+ * library's own). Every wait inside the library's kernels is bounded: when one
+ * runs out the kernel records MFA_ERR_TIMEOUT in the status word, skips the
+ * work that depended on it and returns, so the context stays usable. This call
+ * makes such a wait run out on purpose without any fault: it launches the
+ * decode call's combine kernel alone, on `stream`, for one split sequence whose
+ * partial outputs no attention kernel will ever publish (its flags live in a
+ * small fixed device array of the library that nothing sets), with the waits
+ * limited to wait_ns (1 .. 10^10). It allocates nothing. Returns MFA_OK once
+ * launched (or MFA_ERR_INVALID_ARG / MFA_ERR_CUDA); the kernel then ends after
+ * about wait_ns, and mfa_read_status reports MFA_ERR_TIMEOUT.
+ */
+int mfa_selftest_wait_timeout(unsigned long long wait_ns, mfa_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char* mfa_error_string(int code);

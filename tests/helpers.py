@@ -2,12 +2,13 @@
 run the oracle on the same inputs, and the tolerances used to compare them.
 
 Tolerances (floating point; integer/index work is compared bit-exactly):
-  * bf16 KV cache, fp32 output: max |err| <= 2e-3 on unit-scale outputs (the
-    target stated for this operation). The kernel rounds softmax probabilities to
-    bf16 (relative 2^-9) before the PV product, which bounds its error by
-    2^-9 * max_t |V[t]|; for very short sequences (L < 64) whose outputs are not
-    averaged down that bound can exceed 2e-3, so there the tolerance is
-    max(2e-3, 2^-8 * max_t |V[t]|).
+  * bf16 KV cache, fp32 output: max |err| <= 2e-3 at every sequence length (the
+    target stated for this operation on unit-scale outputs). The kernel carries
+    the softmax probabilities into the PV product as a bf16 pair hi + lo
+    (~16 significant bits), so its error is far below that bound even where a
+    few tokens carry all the weight.
+  * FP8 (E4M3) KV cache: max |err| <= 3e-2 against the oracle on the
+    dequantised cache.
   * bf16 output adds the output rounding, 2^-8 * |ref|.
   * lse: 1e-4 + 1e-5 |lse| (fp32 row sums, hardware exp2/log2).
   * query projection: 2^-8 |ref| (one bf16 rounding of the result) plus
@@ -60,39 +61,22 @@ def oracle_decode(dec: gen.DecodeInputs, select=None):
                       select=select)
 
 
-def v_absmax_per_seq(dec: gen.DecodeInputs) -> np.ndarray:
-    """max_t |V_b[t]| over each sequence's valid rows (dequantised)."""
-    out = np.zeros(dec.batch)
-    v = dec.v
-    for b, L in enumerate(dec.seq_lens.tolist()):
-        if L == 0:
-            continue
-        if dec.page_table is None:
-            rows = v[b, :L]
-        else:
-            t = torch.arange(L)
-            rows = v[dec.page_table[b, t // dec.page_size].long(), t % dec.page_size]
-        if dec.kv_dtype == "e4m3":
-            vals = rows.view(torch.float8_e4m3fn).to(torch.float64) * dec.v_scale
-        else:
-            vals = rows.to(torch.float64)
-        out[b] = float(vals.abs().max())
-    return out
-
-
 def decode_atol(dec: gen.DecodeInputs, ref: np.ndarray, out_dtype, base=2e-3, b_index=None):
-    """Per-element absolute tolerance, broadcastable to ref ([B,H,D] or [n,D])."""
-    vmax = v_absmax_per_seq(dec)
-    lens = dec.seq_lens.numpy()
-    per_b = np.where(lens < 64, np.maximum(base, 2.0 ** -8 * vmax), base)
-    if b_index is not None:
-        tol = per_b[np.asarray(b_index)][:, None]
-    else:
-        tol = per_b[:, None, None]
-    tol = np.broadcast_to(tol, ref.shape).copy()
+    """Per-element absolute tolerance, the shape of ref ([B,H,D] or [n,D]): `base`
+    everywhere, plus one bf16 rounding of the result for bf16 outputs."""
+    tol = np.full(ref.shape, base)
     if out_dtype == torch.bfloat16:
         tol = tol + 2.0 ** -8 * np.abs(ref)
     return tol
+
+
+def max_err_by_length(dec: gen.DecodeInputs, got: np.ndarray, ref: np.ndarray) -> dict:
+    """{sequence length: max |got - ref| over its outputs} (reported by the tests)."""
+    out = {}
+    for b, L in enumerate(dec.seq_lens.tolist()):
+        e = float(np.max(np.abs(got[b] - ref[b])))
+        out[L] = max(out.get(L, 0.0), e)
+    return out
 
 
 def assert_close(got, ref, atol, what=""):

@@ -56,3 +56,46 @@ def test_single_rank_needs_no_process_group():
     assert bench.dist_max(3.5, 1) == 3.5
     bench.barrier(1)
     assert bench.weak_scaling_value(100, 4, 1, 2.0) == 200.0
+
+
+def _stub_runner(args, world, rank, local):
+    """One rank's work with the GPU part left out: the same timing reduction
+    and output rule (rank 0 prints) as the benchmark, over gloo on CPU."""
+    import json
+    import bench
+    assert torch.distributed.get_backend() == "gloo"
+    assert torch.distributed.get_world_size() == args.gpus == world
+    bench.barrier(world)
+    t_max = bench.dist_max(1.0 + rank, world)
+    value = bench.weak_scaling_value(262144, args.steps, world, t_max)
+    bench.barrier(world)
+    if rank == 0:
+        with open(os.environ["MFA_TEST_OUT"], "w") as f:
+            json.dump({"n_gpus": world, "t_max": t_max, "value": value, "rank": rank,
+                       "local": local}, f)
+
+
+def test_bench_launches_its_own_ranks(tmp_path, monkeypatch):
+    """`bench.py --gpus 2` outside torchrun spawns two ranks itself; each joins
+    the process group and rank 0 reports the job-wide figures."""
+    import json
+    import bench
+    out = tmp_path / "line.json"
+    monkeypatch.setenv("MFA_TEST_OUT", str(out))
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    bench.main(["--gpus", "2", "--steps", "10"], runner=_stub_runner)
+    line = json.loads(out.read_text())
+    assert line["n_gpus"] == 2 and line["t_max"] == 2.0 and line["local"] == 0
+    assert line["value"] == pytest.approx(262144 * 10 * 2 / 2.0)
+
+
+def test_bench_single_gpu_runs_in_process(monkeypatch):
+    import bench
+    seen = {}
+
+    def runner(args, world, rank, local):
+        seen.update(world=world, rank=rank, local=local, gpus=args.gpus)
+
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    bench.main(["--gpus", "1"], runner=runner)
+    assert seen == {"world": 1, "rank": 0, "local": 0, "gpus": 1}

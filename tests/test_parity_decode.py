@@ -1,7 +1,8 @@
 """GPU parity of MFA decode attention (bf16 KV cache) against the float64 oracle,
-through the C ABI. Small cases are compared element by element and span
-several 128-token tiles with ragged tails; the full-size workloads are compared
-on sampled (sequence, head) outputs."""
+through the C ABI. Every case compares every output element: small cases span
+several 128-token tiles with ragged tails, and the full-size workloads run in
+the launch configuration the benchmark times. The bound is 2e-3 on fp32
+outputs at every sequence length (plus one bf16 rounding for bf16 outputs)."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +10,8 @@ import torch
 from decode_attention_08_b200 import inputs as gen
 from decode_attention_08_b200 import mfa
 
-from helpers import (assert_close, decode_atol, oracle_decode, run_decode, sample_pairs, to_dev)
+from helpers import (assert_close, decode_atol, max_err_by_length, oracle_decode, run_decode,
+                     to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,8 +33,43 @@ def test_ragged_contiguous_all_outputs(out_dtype):
     dec = gen.make_decode_inputs(102, len(RAGGED), RAGGED, lmax=520)
     got, lse = run_decode(dec, out_dtype=out_dtype, lse=True)
     ref, lref = oracle_decode(dec)
+    print("max |err| by length:", {L: f"{e:.2e}" for L, e in max_err_by_length(dec, got, ref).items()})
     assert_close(got, ref, decode_atol(dec, ref, out_dtype), "out")
     assert_close(lse, lref, 1e-4 + 1e-5 * np.abs(lref), "lse")
+
+
+def test_short_sequences_every_length():
+    """Lengths 1..64, where a few tokens carry all of the softmax weight: the
+    probabilities' precision decides the error here (2e-3 at every length)."""
+    lens = list(range(1, 65))
+    errs = {}
+    for seed in (120, 121):
+        dec = gen.make_decode_inputs(seed, len(lens), lens, lmax=64)
+        got = run_decode(dec)
+        ref, _ = oracle_decode(dec)
+        for L, e in max_err_by_length(dec, got, ref).items():
+            errs[L] = max(errs.get(L, 0.0), e)
+        assert_close(got, ref, decode_atol(dec, ref, torch.float32), f"short, seed {seed}")
+    print("max |err| by length:", {L: f"{e:.2e}" for L, e in errs.items()})
+
+
+def test_concentrated_weights():
+    """Two keys share almost all the weight (q aligned with both) and their
+    values are far apart: rounding the probabilities to bf16 alone gives errors
+    of several 1e-3 here (4.6e-3 at L = 2 in a float64 simulation of it)."""
+    lens = [2, 3, 130, 1000]
+    dec = gen.make_decode_inputs(122, len(lens), lens, lmax=1000)
+    for b, L in enumerate(lens):
+        k0 = dec.k[b, 0].float()
+        k1 = dec.k[b, L - 1].float()
+        dec.q[b] = ((k0 + k1) * (6.0 / 16.0)).to(torch.bfloat16)[None, :].expand(64, 256)
+        dec.q[b, 1::2] = (dec.q[b, 1::2].float() * 1.001).to(torch.bfloat16)
+        dec.v[b, 0] = (torch.sign(dec.v[b, 0].float()) * 4).to(torch.bfloat16)
+        dec.v[b, L - 1] = -dec.v[b, 0]
+    got = run_decode(dec)
+    ref, _ = oracle_decode(dec)
+    err = assert_close(got, ref, decode_atol(dec, ref, torch.float32), "concentrated")
+    print(f"concentrated weights: max |err| {err:.2e}")
 
 
 def test_plain_entry_point_matches_ex():
@@ -148,34 +185,29 @@ def test_length_beyond_cache_is_reported():
     assert mfa.read_status() == mfa.STATUS_CODES["MFA_ERR_BAD_INDEX"]
 
 
-# ---- the five workloads at full size (sampled outputs) -----------------------
+# ---- the workloads at full size, every output ------------------------------
 
-def _full_workload_check(index, nsample, num_splits=0):
+def _full_workload_check(index, num_splits=0):
     dec, _ = gen.make_workload(index)
     got = run_decode(dec, num_splits=num_splits)
     assert np.all(np.isfinite(got))
-    pairs = sample_pairs(dec.batch, nsample, 900 + index)
-    ref, _ = oracle_decode(dec, select=pairs)
-    bi = [b for b, _ in pairs]
-    g = np.stack([got[b, h] for b, h in pairs])
-    return assert_close(g, ref, decode_atol(dec, ref, torch.float32, b_index=bi),
-                        gen.WORKLOADS[index]["name"])
+    ref, _ = oracle_decode(dec)
+    err = assert_close(got, ref, decode_atol(dec, ref, torch.float32), gen.WORKLOADS[index]["name"])
+    print(f"{gen.WORKLOADS[index]['name']}: max |err| {err:.2e} over {got.size} outputs")
+    return err
 
 
 def test_workload1_all_outputs():
-    dec, _ = gen.make_workload(1)
-    got = run_decode(dec)
-    ref, _ = oracle_decode(dec)
-    assert_close(got, ref, decode_atol(dec, ref, torch.float32), "workload 1")
+    _full_workload_check(1)
 
 
-def test_workload2_sampled():
-    _full_workload_check(2, 48)
+def test_workload2_all_outputs():
+    _full_workload_check(2)
 
 
-def test_workload3_paged_sampled():
-    _full_workload_check(3, 48)
+def test_workload3_paged_all_outputs():
+    _full_workload_check(3)
 
 
-def test_workload5_attention_split16_sampled():
-    _full_workload_check(5, 24, num_splits=16)
+def test_workload5_attention_split16_all_outputs():
+    _full_workload_check(5, num_splits=16)

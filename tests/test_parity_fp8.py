@@ -1,9 +1,10 @@
 """GPU parity of MFA decode attention over an FP8 E4M3 KV cache with per-tensor
 scales, against the float64 oracle on the dequantised cache, through the C ABI.
 
-Tolerance: max |err| <= 3e-2 (the stated FP8-KV target). The kernel expands the
-codes exactly to f16 and runs f16 x f16 products with fp32 accumulation, so its
-error is that of the bf16 path or smaller; the test also reports it.
+Tolerance: max |err| <= 3e-2 (the stated FP8-KV target) at every length. The
+kernel runs E4M3 x E4M3 tensor-core products (kind::f8f6f4) straight from the
+cache, with q and the probabilities entering as exact E4M3 pairs hi + lo, so
+its error stays at the level of the bf16 path; the tests report it.
 """
 import numpy as np
 import pytest
@@ -12,7 +13,7 @@ import torch
 from decode_attention_08_b200 import inputs as gen
 from decode_attention_08_b200 import mfa
 
-from helpers import assert_close, decode_atol, oracle_decode, run_decode, sample_pairs
+from helpers import assert_close, decode_atol, max_err_by_length, oracle_decode, run_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +44,7 @@ def test_fp8_ragged_contiguous(out_dtype):
     dec = gen.make_decode_inputs(502, len(lens), lens, lmax=4100, kv_dtype="e4m3")
     got, lse = run_decode(dec, out_dtype=out_dtype, lse=True)
     ref, lref = oracle_decode(dec)
+    print("max |err| by length:", {L: f"{e:.2e}" for L, e in max_err_by_length(dec, got, ref).items()})
     err = assert_close(got, ref, decode_atol(dec, ref, out_dtype, base=FP8_TOL), "fp8 out")
     assert_close(lse, lref, 1e-4 + 1e-5 * np.abs(lref), "fp8 lse")
     assert err < FP8_TOL
@@ -78,12 +80,10 @@ def test_fp8_fixed_splits():
     assert_close(got, ref, decode_atol(dec, ref, torch.float32, base=FP8_TOL), "fp8 splits")
 
 
-def test_workload4_fp8_sampled():
+def test_workload4_fp8_all_outputs():
     dec, _ = gen.make_workload(4)
     got = run_decode(dec)
     assert np.all(np.isfinite(got))
-    pairs = sample_pairs(dec.batch, 48, 904)
-    ref, _ = oracle_decode(dec, select=pairs)
-    g = np.stack([got[b, h] for b, h in pairs])
-    bi = [b for b, _ in pairs]
-    assert_close(g, ref, decode_atol(dec, ref, torch.float32, base=FP8_TOL, b_index=bi), "wl4")
+    ref, _ = oracle_decode(dec)
+    err = assert_close(got, ref, decode_atol(dec, ref, torch.float32, base=FP8_TOL), "wl4")
+    print(f"workload 4: max |err| {err:.2e} over {got.size} outputs")

@@ -57,3 +57,13 @@ def test_step3_shape_batch8():
     got = _run(p)
     ref = _ref(p)
     assert_close(got, ref, _tol(ref), "step3")
+
+
+@pytest.mark.parametrize("batch", [16, 64])
+def test_step3_shape_two_launch_path(batch):
+    """Batches above 8 take the two-launch path (split-K latent GEMM, then the
+    up-projection); checked at the Step-3 shapes on every output."""
+    p = gen.make_proj_inputs(2100 + batch, batch)
+    got = _run(p)
+    ref = _ref(p)
+    assert_close(got, ref, _tol(ref), f"step3 batch {batch}")

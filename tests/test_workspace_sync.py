@@ -1,14 +1,15 @@
-"""GPU tests of the decode workspace's synchronisation words.
+"""GPU tests of the decode workspace's hand-off between the call's two kernels.
 
 The combine kernel starts while the attention kernel still runs and merges a
-split sequence once the last writer of its partials has arrived. The words
-that carry this (an arrival counter and four ready words per sequence) sit at
-the start of the caller's workspace; every call returns them to zero, and the
-library clears them when a workspace is new to it or serves another batch size.
+split sequence once the flags of all its partial slots are set. Every word it
+reads (the per-sequence plan words, the per-slot flags) is written by the
+attention kernel of the same call before the combine kernel may start, so a
+workspace needs no initialisation and nothing left in it by an earlier call,
+of any shape, or by anything else, can change a result.
 
-Each test compares against a call on a fresh zero-filled workspace, which the
-parity tests tie to the oracle; results must be bit-identical, because the
-split plan (and so the arithmetic) does not depend on the workspace.
+Each test compares against a call on a fresh workspace, which the parity tests
+tie to the oracle; results must be bit-identical, because the split plan (and
+so the arithmetic) does not depend on the workspace.
 """
 import numpy as np
 import pytest
@@ -33,15 +34,6 @@ def _fresh(dec, num_splits=0):
     return run_decode(dec, num_splits=num_splits)
 
 
-def _sync_words(ws, batch):
-    """Arrival counters [B] (u32) and ready words [B][4] (u64) of a workspace."""
-    raw = ws.cpu().numpy()
-    arrive = raw[:4 * batch].view(np.uint32)
-    ready_off = (4 * batch + 15) & ~15
-    ready = raw[ready_off:ready_off + 32 * batch].view(np.uint64)
-    return arrive, ready
-
-
 def _mixed(seed, batch, lmax):
     rng = np.random.default_rng(seed)
     lens = rng.integers(0, lmax + 1, size=batch).tolist()
@@ -49,16 +41,63 @@ def _mixed(seed, batch, lmax):
     return gen.make_decode_inputs(seed, batch, lens, lmax=lmax)
 
 
-def test_sync_words_are_zero_after_each_call():
+def _garbage(ws, kind, seed=0):
+    """Fill a workspace with a pattern a caller's memory might hold."""
+    if kind == "random":
+        g = torch.Generator(device="cuda").manual_seed(seed)
+        ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda", generator=g))
+    elif kind == "ones":
+        ws.fill_(0xFF)
+    elif kind == "small_ints":  # words of 1: every flag "set"
+        ws.view(torch.int32).fill_(1)
+    else:
+        ws.zero_()
+
+
+@pytest.mark.parametrize("kind", ["random", "ones", "small_ints"])
+@pytest.mark.parametrize("num_splits", [0, 5])
+def test_garbage_filled_workspace(kind, num_splits):
     dec = _mixed(601, 40, 6000)
+    want = _fresh(dec, num_splits)
     t = to_dev(dec)
-    ws = torch.zeros(mfa.decode_workspace_size(dec.batch, 0), dtype=torch.uint8, device="cuda")
-    out = torch.empty(dec.batch, 64, 256, dtype=torch.float32, device="cuda")
-    for _ in range(3):
-        _call(t, dec, out, ws)
+    ws = torch.empty(mfa.decode_workspace_size(dec.batch, num_splits), dtype=torch.uint8,
+                     device="cuda")
+    for i in range(2):
+        _garbage(ws, kind, seed=i)
+        out = torch.full((dec.batch, 64, 256), float("nan"), dtype=torch.float32, device="cuda")
+        _call(t, dec, out, ws, num_splits)
         assert mfa.read_status() == 0
-        arrive, ready = _sync_words(ws, dec.batch)
-        assert not arrive.any() and not ready.any()
+        assert np.array_equal(out.double().cpu().numpy(), want), (kind, i)
+
+
+def test_workspace_freed_and_reallocated_at_the_same_address():
+    """A caching allocator hands a freed block back at the same address with
+    whatever it last held: here the words another call (another batch size)
+    left, then random bytes. No memset in between."""
+    a = _mixed(602, 64, 5000)
+    b = _mixed(603, 5, 9000)
+    want_a, want_b = _fresh(a), _fresh(b)
+    ta, tb = to_dev(a), to_dev(b)
+    need = max(mfa.decode_workspace_size(64, 0), mfa.decode_workspace_size(5, 0))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    addr = ws.data_ptr()
+    out_a = torch.empty(64, 64, 256, dtype=torch.float32, device="cuda")
+    _call(ta, a, out_a, ws)
+    assert mfa.read_status() == 0
+    del ws
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")  # same block, contents kept
+    out_b = torch.full((5, 64, 256), float("nan"), dtype=torch.float32, device="cuda")
+    _call(tb, b, out_b, ws)
+    assert mfa.read_status() == 0
+    assert np.array_equal(out_b.double().cpu().numpy(), want_b)
+    del ws
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    _garbage(ws, "random", seed=7)
+    out_a.fill_(float("nan"))
+    _call(ta, a, out_a, ws)
+    assert mfa.read_status() == 0
+    assert np.array_equal(out_a.double().cpu().numpy(), want_a)
+    print("same address reused:", ws.data_ptr() == addr)
 
 
 def test_one_workspace_across_batch_sizes_and_split_modes():
@@ -73,7 +112,8 @@ def test_one_workspace_across_batch_sizes_and_split_modes():
     }
     need = max(mfa.decode_workspace_size(d.batch, s)
                for d, s in ((big, 0), (small, 0), (small, 3), (paged, 0)))
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    _garbage(ws, "random", seed=3)
     tens = {"big": (big, to_dev(big)), "small": (small, to_dev(small)),
             "paged": (paged, to_dev(paged))}
     order = [("big", 0), ("small", 0), ("big", 0), ("small", 3), ("paged", 0), ("small", 0),
@@ -92,7 +132,7 @@ def test_back_to_back_calls_without_host_sync():
     b = _mixed(606, 32, 3000)
     want_a, want_b = _fresh(a), _fresh(b)
     ta, tb = to_dev(a), to_dev(b)
-    ws = torch.zeros(mfa.decode_workspace_size(32, 0), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(mfa.decode_workspace_size(32, 0), dtype=torch.uint8, device="cuda")
     outs = [torch.empty(32, 64, 256, dtype=torch.float32, device="cuda") for _ in range(12)]
     for i, out in enumerate(outs):
         dec, t = (a, ta) if i % 2 == 0 else (b, tb)
@@ -107,11 +147,10 @@ def test_back_to_back_calls_without_host_sync():
 def test_graph_replays(calls_per_graph):
     dec = _mixed(607, 48, 6000)
     t = to_dev(dec)
-    ws = torch.zeros(mfa.decode_workspace_size(dec.batch, 0), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(mfa.decode_workspace_size(dec.batch, 0), dtype=torch.uint8, device="cuda")
+    _garbage(ws, "ones")
     out = torch.empty(dec.batch, 64, 256, dtype=torch.float32, device="cuda")
     st = torch.cuda.Stream()
-    with torch.cuda.stream(st):
-        _call(t, dec, out, ws, stream=st)  # first sight of the workspace: outside capture
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=st):

@@ -67,6 +67,46 @@ def test_noalloc_paged_fixed_splits_matches_workspace_entry_point():
     _check_two_calls(gen.make_decode_inputs(402, len(lens), lens, page_size=64), num_splits=4)
 
 
+def test_noalloc_allocates_no_device_memory():
+    """After a first call (which looks up the array's address), further calls
+    change neither the device's free memory nor torch's allocations."""
+    lens = [4096, 17, 2000, 0, 5000]
+    dec = gen.make_decode_inputs(404, len(lens), lens)
+    t = to_dev(dec)
+    out = torch.empty(dec.batch, 64, 256, dtype=torch.float32, device="cuda")
+    assert _noalloc(t, dec, out) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for splits in (0, 3):
+        assert _noalloc(t, dec, out, None, splits) == 0
+    torch.cuda.synchronize()
+    assert mfa.read_status() == 0
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0 and torch.cuda.memory_allocated() == alloc0
+
+
+def test_noalloc_fp8_through_the_python_wrapper():
+    """FP8 cache with per-tensor scales, through mfa.decode_attention_noalloc,
+    twice in a row, against mfa.decode_attention_ex (3e-2, the FP8 bound)."""
+    lens = [4096, 1, 300, 2500]
+    dec = gen.make_decode_inputs(405, len(lens), lens, kv_dtype="e4m3")
+    t = to_dev(dec)
+    want = torch.empty(dec.batch, 64, 256, dtype=torch.float32, device="cuda")
+    mfa.decode_attention_ex(t["q"], t["k"], t["v"], None, t["seq_lens"], want,
+                            dec.softmax_scale, "e4m3", k_scale=dec.k_scale, v_scale=dec.v_scale)
+    assert mfa.read_status() == 0
+    want = want.double().cpu().numpy()
+    for _ in range(2):
+        got = torch.full((dec.batch, 64, 256), float("nan"), dtype=torch.float32, device="cuda")
+        mfa.decode_attention_noalloc(t["q"], t["k"], t["v"], None, t["seq_lens"], got,
+                                     dec.softmax_scale, "e4m3", k_scale=dec.k_scale,
+                                     v_scale=dec.v_scale)
+        assert mfa.read_status() == 0
+        got = got.double().cpu().numpy()
+        assert_close(got, want, decode_atol(dec, want, torch.float32, base=3e-2), "fp8 noalloc")
+
+
 def test_noalloc_rejects_requests_beyond_its_array():
     # 400 sequences x 1024 splits needs far more than the fixed 24 MiB array
     dec = gen.make_decode_inputs(403, 400, 1)
