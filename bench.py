@@ -50,7 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle's CPU-baseline sample")
-    ap.add_argument("--profile", choices=["decode", "paged", "fp8", "qproj", "lse_merge"],
+    ap.add_argument("--profile", choices=["decode", "paged", "fp8", "qproj", "lse_merge", "gqa",
+                                          "out_proj", "kv_append", "fused"],
                     default=None,
                     help="profiling case for ncu: plain launches of one kernel family on a "
                          "reduced workload that still exceeds L2")
@@ -898,6 +899,32 @@ def run_profile_case(args):
         q = torch.empty(8, wb.shape[1], dtype=torch.bfloat16, device="cuda")
         for _ in range(args.warmup + args.steps):
             mfa.query_proj(x, wa, wb, q)
+    elif args.profile == "out_proj":
+        inp = gen.make_out_proj_inputs(4008, 8)
+        o, wo = inp.o.cuda(), inp.w_o.cuda()
+        y = torch.empty(8, wo.shape[1], dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(mfa.output_proj_workspace_size(8, o.shape[1], wo.shape[1]),
+                         dtype=torch.uint8, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            mfa.output_proj(o, wo, y, ws)
+    elif args.profile == "kv_append":
+        inp = gen.make_kv_append_inputs(3064, 64)
+        x, wk, wv = inp.x.cuda(), inp.w_k.cuda(), inp.w_v.cuda()
+        kc = torch.zeros(64, 4096, 256, dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        pos = torch.full((64,), 4000, dtype=torch.int32, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            mfa.kv_append(x, wk, wv, kc, vc, pos)
+    elif args.profile == "gqa":
+        inp = gen.make_gqa_inputs(1100, 48, 4096)
+        step = GqaStep(inp, copies=1)
+        for i in range(args.warmup + args.steps):
+            step.call(i)
+    elif args.profile == "fused":
+        dec, proj = gen.make_workload(5)
+        step = FusedStep(dec, proj, 1, dec.meta.get("num_splits", 0))
+        for i in range(args.warmup + args.steps):
+            step.call(i)
     else:
         if args.profile == "decode":
             dec = gen.make_decode_inputs(1002, 48, 4096)

@@ -113,9 +113,6 @@ struct __align__(16) DecodeCtrl {
   unsigned qmax[Geo<kFp8>::kQGroupWarps];  // FP8: per-warp max |q| bits, first segment's conversion
   int b_start, off_start, tiles;
   int scan_warp[Geo<kFp8>::kThreads / 32];
-  // balanced plan: lens[0] = b_start, lens[1 + k] = validated length of
-  // sequence b_start + k (k < 8)
-  int lens[9];
   // vector-loaded (float4): keep 16-byte aligned
   // [tile parity][warpgroup][warp][head]: per-warp tile maxima; at a
   // segment's end the same buffer carries the per-warp row sums
@@ -236,7 +233,6 @@ struct TileStream {
   // never reloads them through memory (the hot loops hold memory-clobbering
   // waits, after which a pointer read would go back out to the cache hierarchy)
   const int* seq_lens;
-  const int* lens;  // shared copy of some lengths ({first sequence, 8 lengths}), or nullptr
   int cap_tokens, num_splits, grid, batch;
   int cta;
   int b, tile, L, nt, remaining, seg_lo, seg_hi, seg_ord;
@@ -244,10 +240,9 @@ struct TileStream {
   long long gtile;
   int unit, unit_hi;
 
-  __device__ void init(const DecodeParams& prm, const int* lens_, int b_start, int off_start,
-                       int tiles, long long t0) {
+  __device__ void init(const DecodeParams& prm, int b_start, int off_start, int tiles,
+                       long long t0) {
     seq_lens = prm.seq_lens;
-    lens = prm.num_splits == 0 ? lens_ : nullptr;
     cap_tokens = prm.cap_tokens;
     num_splits = prm.num_splits;
     grid = prm.grid;
@@ -274,11 +269,9 @@ struct TileStream {
   }
 
   // fixed plan: move to the next non-empty unit owned by this CTA
+  // (a global load: a shared copy of the lengths costs the FP8 kernel registers
+  // it does not have, and reaches only a few loads per CTA)
   __device__ int length(int seq) const {
-    if (lens) {
-      const unsigned k = static_cast<unsigned>(seq - lens[0]);
-      if (k < 8u) return lens[1 + k];
-    }
     int n = __ldg(seq_lens + seq);
     if (n < 0 || n > cap_tokens) {
       record_error(5 /* MFA_ERR_BAD_INDEX */);
@@ -960,7 +953,8 @@ __device__ __noinline__ void segment_out(float* ws_o, void* out, int out_f32, in
     } else {
       tmem_wait_ld();
     }
-    // per head j: the output scale held by lane j
+    // per head j: the output scale held by lane j (a shuffle; a shared-memory
+    // copy measured slower: it cost the 168-register kernel a spill)
 #pragma unroll
     for (int j = 0; j < W; ++j)
       r[j] = __float_as_uint(__uint_as_float(r[j]) * __shfl_sync(0xffffffffu, ev, j));
@@ -1096,17 +1090,12 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
       g_mfa_gt[((gt_call * 2) * kGtCtas + blockIdx.x) * 3] = gt_start;
   }
 #endif
-  // balanced plan: the tile streams find the lengths of this CTA's first eight
-  // sequences in shared memory (others in global memory)
-  const int* lens_s = c.lens;
   if (p.num_splits == 0) {
     balanced_plan(p, c);  // ends with __syncthreads
     if (tid == 0) {  // the next call's L2 warm-up hint
       p.ws_hint[2 * blockIdx.x] = c.tiles > 0 ? c.b_start : -1;
       p.ws_hint[2 * blockIdx.x + 1] = c.off_start;
     }
-    if (tid < 8) c.lens[1 + tid] = c.b_start + tid < p.batch ? valid_len(p, c.b_start + tid) : 0;
-    if (tid == 8) c.lens[0] = c.b_start;
   } else if (tid == 0) {
     c.tiles = static_cast<int>(blockIdx.x) < p.batch * p.num_splits ? -1 : 0;
     c.t0 = 0;
@@ -1140,7 +1129,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     // ======================= K/V producer ===================================
     const uint64_t policy = l2_policy_evict_first();
     TileStream ks;
-    ks.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    ks.init(p, c.b_start, c.off_start, c.tiles, c.t0);
     uint32_t item = 0;
 #ifdef MFA_TRACE
     int ntr[2] = {0, 0};
@@ -1269,23 +1258,25 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     const uint32_t ring_base = smem_u32(sRing);
     const uint32_t p_base = smem_u32(sP);
     TileStream qs;
-    qs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
-    uint32_t item = 0, nq = 0;
+    qs.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+    uint32_t nq = 0;
     bool ok = true;
-    // waits for the kIPT ring items of the next tensor; returns the first
-    auto take_items = [&](uint32_t& first) -> bool {
-      first = item;
-      item += kIPT;
+    // Ring items, in the producer's order K0 | K1 V0 | K2 V1 | ... | V(T-1),
+    // kIPT per tensor: the first item of K(j) and of V(j) (the CTA's j-th tile).
+    auto k_item = [](uint32_t j) -> uint32_t { return j == 0 ? 0u : (2u * j - 1u) * kIPT; };
+    auto v_first = [](uint32_t j, bool cta_last) -> uint32_t {
+      return (cta_last ? 2u * j + 1u : 2u * j + 2u) * kIPT;
+    };
+    // every lane tests (each acquires on success); the warp agrees
+    auto items_ready = [&](uint32_t first) -> bool {
+      bool r = true;
       for (uint32_t u = 0; u < kIPT; ++u)
-        if (!mbar_wait_warp(&c.slot_full[(first + u) % kS], par((first + u) / kS), abort_flag))
-          return false;
-      return true;
+        r = r && mbar_test_wait(&c.slot_full[(first + u) % kS], par((first + u) / kS));
+      return __all_sync(0xffffffffu, r);
     };
 
-    auto issue_pv = [&](const TileInfo& t, uint32_t j) -> bool {
-      if (!mbar_wait_warp(&c.p_full, par(j), abort_flag)) return false;
-      uint32_t lo;
-      if (!take_items(lo)) return false;
+    auto issue_pv = [&](const TileInfo& t, uint32_t j) {
+      const uint32_t lo = v_first(j, t.cta_last);
       tc_fence_after();
       if (lane == 0) MFA_TR(3, j);
       // the whole warp issues (one elected lane; see mma_f16_ss_warp)
@@ -1327,27 +1318,13 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
         mma_commit_warp(&c.slot_empty[hi % kS]);
       }
       mma_commit_warp(&c.o_full);
-      return true;
     };
 
-    TileInfo cur, prev;
-    uint32_t g = 0;
-    uint32_t qbuf = 0;  // q buffer of the current segment
-    while (ok && qs.next(cur)) {
-      if (cur.seg_first) {
-        // segment nq uses q buffer nq & 1 (FP8) or the only one (bf16)
-        qbuf = kFp8 ? (nq & 1u) : 0u;
-        ok = mbar_wait_warp(kFp8 ? &c.q_conv[qbuf] : &c.q_full[0], kFp8 ? par(nq >> 1) : par(nq),
-                       abort_flag);
-        ++nq;
-        if (!ok) break;
-      }
-      if (g >= 2 && !(ok = mbar_wait_warp(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag))) break;
-      uint32_t lo;
-      if (!(ok = take_items(lo))) break;
+    auto issue_qk = [&](const TileInfo& t, uint32_t j, uint32_t qbuf) {
+      const uint32_t lo = k_item(j);
       tc_fence_after();
-      if (lane == 0) MFA_TR(2, g);
-      const uint32_t d_s = tmem + s_cols<kFp8>(g);
+      if (lane == 0) MFA_TR(2, j);
+      const uint32_t d_s = tmem + s_cols<kFp8>(j);
       if (kFp8) {
         // K slot: head dims 0-127 | 128-255 (128 token rows of 128 B, K-major);
         // q: per dims half, the 64 hi rows then the 64 lo rows (128 B each,
@@ -1379,13 +1356,88 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
         mma_commit_warp(&c.slot_empty[lo % kS]);
         mma_commit_warp(&c.slot_empty[hi % kS]);
       }
-      mma_commit_warp(&c.s_full[g & 1]);
-      if (cur.seg_last) mma_commit_warp(&c.q_empty[qbuf]);
-      if (g >= 1 && !(ok = issue_pv(prev, g - 1))) break;
-      prev = cur;
-      ++g;
+      mma_commit_warp(&c.s_full[j & 1]);
+      if (t.seg_last) mma_commit_warp(&c.q_empty[qbuf]);
+    };
+
+    // Each round issues the scores of tile g and the PV product of tile g - 1,
+    // in that order. With an FP8 cache, while both are pending, the warp polls
+    // both and issues whichever has its inputs first, the scores preferred (the
+    // softmax needs S(g) before it needs PV(g - 1) done), so the PV product does
+    // not wait behind a late K tile; the one left is then awaited as before.
+    // (Measured: FP8 workload 72.8 -> 71.8 us; with a bf16 cache the polling
+    // warp slowed the HBM-bound pipeline, 54.4 -> 57.6 us, so it keeps the
+    // plain order.) Every wait is bounded.
+    auto wait_items = [&](uint32_t first) -> bool {
+      for (uint32_t u = 0; u < kIPT; ++u)
+        if (!mbar_wait_warp(&c.slot_full[(first + u) % kS], par((first + u) / kS), abort_flag))
+          return false;
+      return true;
+    };
+    TileInfo cur, prev;
+    uint32_t g = 0;
+    uint32_t qbuf = 0;  // q buffer of the current segment
+    bool have_cur = qs.next(cur), pending_pv = false;
+    while (ok && (have_cur || pending_pv)) {
+      bool need_qk = have_cur, need_pv = pending_pv;
+      if (have_cur && cur.seg_first) qbuf = kFp8 ? (nq & 1u) : 0u;
+      uint64_t* qbar = kFp8 ? &c.q_conv[qbuf] : &c.q_full[0];
+      const uint32_t qpar = kFp8 ? par(nq >> 1) : par(nq);
+      if (kFp8 && need_qk && need_pv) {
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t spin = 1;; ++spin) {
+          if ((!cur.seg_first || __all_sync(0xffffffffu, mbar_test_wait(qbar, qpar))) &&
+              (g < 2 || __all_sync(0xffffffffu,
+                                   mbar_test_wait(&c.s_empty[g & 1], par((g >> 1) - 1)))) &&
+              items_ready(k_item(g))) {
+            issue_qk(cur, g, qbuf);
+            need_qk = false;
+            break;
+          }
+          if (__all_sync(0xffffffffu, mbar_test_wait(&c.p_full, par(g - 1))) &&
+              items_ready(v_first(g - 1, prev.cta_last))) {
+            issue_pv(prev, g - 1);
+            need_pv = false;
+            break;
+          }
+          if ((spin & 255u) == 0) {
+            bool stop = *abort_flag != 0;
+            if (!stop && global_timer_ns() - t0 > kWaitLimitNs) {
+              if (lane == 0) {
+                record_error(6 /* MFA_ERR_TIMEOUT */);
+                *abort_flag = 1;
+              }
+              stop = true;
+            }
+            if (__any_sync(0xffffffffu, stop)) {
+              ok = false;
+              break;
+            }
+          }
+        }
+      }
+      if (ok && need_qk) {
+        ok = (!cur.seg_first || mbar_wait_warp(qbar, qpar, abort_flag)) &&
+             (g < 2 || mbar_wait_warp(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag)) &&
+             wait_items(k_item(g));
+        if (ok) issue_qk(cur, g, qbuf);
+      }
+      if (ok && need_pv) {
+        ok = mbar_wait_warp(&c.p_full, par(g - 1), abort_flag) &&
+             wait_items(v_first(g - 1, prev.cta_last));
+        if (ok) issue_pv(prev, g - 1);
+      }
+      if (!ok) break;
+      if (have_cur) {
+        if (cur.seg_first) ++nq;
+        prev = cur;
+        ++g;
+        pending_pv = true;  // PV of the tile just scored
+        have_cur = qs.next(cur);
+      } else {
+        pending_pv = false;  // this round issued the last tile's PV
+      }
     }
-    if (ok && g >= 1) ok = issue_pv(prev, g - 1);
     if (!ok && lane == 0) {
       // drain: wait (bounded, ignoring the abort flag) for issued MMAs
       mma_commit(&c.drain);
@@ -1403,8 +1455,8 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     // is on its way, since k - 1's last PV is issued after k's first QK.
     const uint64_t policy = l2_policy_evict_last();
     TileStream qs, ahead;
-    qs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
-    ahead.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    qs.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+    ahead.init(p, c.b_start, c.off_start, c.tiles, c.t0);
     TileInfo t, ta, last;
     bool more_ahead = ahead.next(ta);  // stays one segment ahead of qs
     bool have_last = false, ok = true;
@@ -1468,7 +1520,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
       // through a four-entry ring (this warp runs at most two segments ahead
       // of them: q of the next segment waits for the current one's last QK).
       TileStream cs;
-      cs.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+      cs.init(p, c.b_start, c.off_start, c.tiles, c.t0);
       TileInfo t;
       uint32_t nq = 0;
       while (cs.next(t)) {
@@ -1494,7 +1546,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
       // After the softmax warps have written a segment's output or partial,
       // makes it visible device-wide and tells the combine kernel.
       TileStream ns;
-      ns.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+      ns.init(p, c.b_start, c.off_start, c.tiles, c.t0);
       TileInfo t;
       unsigned k = 0;
       while (ns.next(t)) {
@@ -1517,7 +1569,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     const int hl = lane & (kWGHeads - 1);
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
     TileStream ts;
-    ts.init(p, lens_s, c.b_start, c.off_start, c.tiles, c.t0);
+    ts.init(p, c.b_start, c.off_start, c.tiles, c.t0);
     if (kFp8) {
       // the first segment's q conversion, with warp 3 (which publishes it)
       TileStream first = ts;

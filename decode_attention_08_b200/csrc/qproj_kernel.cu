@@ -179,6 +179,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched with programmatic dependent launch: the set-up above may overlap
+  // the previous kernel's tail; nothing in global memory is touched before it
+  // has completed
+  griddep_wait();
   const uint32_t tmem = c.tmem_base;
   volatile int* abort_flag = &c.abort_flag;
 
@@ -369,6 +373,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched with programmatic dependent launch: the set-up above may overlap
+  // the previous kernel's tail; nothing in global memory is touched before it
+  // has completed
+  griddep_wait();
   const uint32_t tmem = c.tmem_base;
   volatile int* abort_flag = &c.abort_flag;
 
@@ -567,6 +575,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kFusedTmemCols);
 }
 
+// Launch with programmatic dependent launch (the kernel waits for the
+// previous kernel on the stream before it touches global memory).
+template <typename Kernel, typename... Args>
+static cudaError_t launch_pdl_qp(Kernel kernel, dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int qproj_fused_smem_bytes(int n1, int n2) {
   const int stage_bytes = fused_stage_bytes(n1, n2);
   return fused_stages(stage_bytes) * stage_bytes + static_cast<int>(sizeof(FusedCtrl)) + 1024;
@@ -584,8 +610,8 @@ cudaError_t launch_qproj_fused(const CUtensorMap& twa, const CUtensorMap& tx,
   cudaError_t err = cudaFuncSetAttribute(mfa_qproj_fused_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  mfa_qproj_fused_kernel<<<grid, kFusedThreads, smem, stream>>>(twa, tx, twb, tl, p);
-  return cudaGetLastError();
+  return launch_pdl_qp(mfa_qproj_fused_kernel, dim3(grid), dim3(kFusedThreads),
+                       static_cast<size_t>(smem), stream, twa, tx, twb, tl, p);
 }
 
 int qproj_smem_bytes(int n_cols) {
@@ -600,7 +626,9 @@ cudaError_t launch_qproj(const CUtensorMap& tw, const CUtensorMap& ta, const Qpr
       cudaFuncSetAttribute(mfa_qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   dim3 grid(m_tiles, p.mode == 1 ? 1 : p.splits);
-  mfa_qproj_kernel<<<grid, kGemmThreads, smem, stream>>>(tw, ta, tw, p);
+  const cudaError_t e = launch_pdl_qp(mfa_qproj_kernel, grid, dim3(kGemmThreads),
+                                      static_cast<size_t>(smem), stream, tw, ta, tw, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
