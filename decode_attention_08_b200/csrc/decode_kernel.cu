@@ -112,6 +112,7 @@ struct __align__(16) DecodeCtrl {
   float qinv[4];          // FP8 cache: score scale 1/s of segment k at [k & 3]
   unsigned qmax[Geo<kFp8>::kQGroupWarps];  // FP8: per-warp max |q| bits, first segment's conversion
   int b_start, off_start, tiles;
+  int L_start;  // length of sequence b_start (balanced plan)
   int scan_warp[Geo<kFp8>::kThreads / 32];
   // vector-loaded (float4): keep 16-byte aligned
   // [tile parity][warpgroup][warp][head]: per-warp tile maxima; at a
@@ -240,8 +241,9 @@ struct TileStream {
   long long gtile;
   int unit, unit_hi;
 
+  // L0: the length of sequence b_start, as the plan read it (balanced plan)
   __device__ void init(const DecodeParams& prm, int b_start, int off_start, int tiles,
-                       long long t0) {
+                       long long t0, int L0) {
     seq_lens = prm.seq_lens;
     cap_tokens = prm.cap_tokens;
     num_splits = prm.num_splits;
@@ -255,7 +257,7 @@ struct TileStream {
       remaining = tiles;
       if (remaining > 0) {
         b = b_start;
-        L = length(b);
+        L = L0;
         nt = tiles_of(L);
         tile = off_start;
         seg_lo = tile;
@@ -483,7 +485,8 @@ __device__ void balanced_plan(const DecodeParams& p, DecodeCtrl<kFp8>& c) {
   long long t0 = 0;
   if (p.batch <= kThreads) {
     // single pass: the whole batch is one chunk
-    const int n = tid < p.batch ? tiles_of(valid_len(p, tid)) : 0;
+    const int len = tid < p.batch ? valid_len(p, tid) : 0;
+    const int n = tiles_of(len);
     int chunk;
     const int incl = block_inclusive_scan<kThreads>(n, c.scan_warp, &chunk);
     total = chunk;
@@ -492,10 +495,13 @@ __device__ void balanced_plan(const DecodeParams& p, DecodeCtrl<kFp8>& c) {
     if (tid < p.batch && n > 0 && excl <= t0 && t0 < excl + n) {
       c.b_start = tid;
       c.off_start = static_cast<int>(t0 - excl);
+      c.L_start = len;
     }
-    if (tid < p.batch && tid % p.grid == static_cast<int>(blockIdx.x))
+    if (tid < p.batch && tid % p.grid == static_cast<int>(blockIdx.x)) {
       p.ws_plan[tid] = static_cast<unsigned long long>(excl) |
                        (static_cast<unsigned long long>(total) << 32);
+      __threadfence();  // before the combine may start (the trigger follows this plan)
+    }
   } else {
     for (int base = 0; base < p.batch; base += kThreads) {
       const int b = base + tid;
@@ -508,17 +514,21 @@ __device__ void balanced_plan(const DecodeParams& p, DecodeCtrl<kFp8>& c) {
     long long run = 0;
     for (int base = 0; base < p.batch; base += kThreads) {
       const int b = base + tid;
-      const int n = (b < p.batch) ? tiles_of(valid_len(p, b)) : 0;
+      const int len = (b < p.batch) ? valid_len(p, b) : 0;
+      const int n = tiles_of(len);
       int chunk;
       const int incl = block_inclusive_scan<kThreads>(n, c.scan_warp, &chunk);
       const long long excl = run + incl - n;
       if (b < p.batch && n > 0 && excl <= t0 && t0 < excl + n) {
         c.b_start = b;
         c.off_start = static_cast<int>(t0 - excl);
+        c.L_start = len;
       }
-      if (b < p.batch && b % p.grid == static_cast<int>(blockIdx.x))
+      if (b < p.batch && b % p.grid == static_cast<int>(blockIdx.x)) {
         p.ws_plan[b] = static_cast<unsigned long long>(excl) |
                        (static_cast<unsigned long long>(total) << 32);
+        __threadfence();  // before the combine may start (the trigger follows this plan)
+      }
       run += chunk;
     }
   }
@@ -782,7 +792,6 @@ __device__ __forceinline__ float q_to_e4m3_group(uint32_t base, int gtid, bool w
 
 constexpr int kCombineHeads = 16;  // heads per CTA
 constexpr int kCombineDims = 16;   // head-dim elements per thread (kDim / 16 threads per head)
-constexpr int kCombineBatch = 4;   // partials loaded per round trip
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* w) {
   unsigned v;
@@ -839,6 +848,8 @@ __device__ __forceinline__ void store_out16(const DecodeParams& p, int b, int h,
 // d0 .. d0 + 15, in plan order (up to four per round trip), and writes the
 // output and (d0 == 0) the log-sum-exp. The partials must be visible to the
 // caller (acquired after the sequence's last arrival).
+// kCombineBatch: partials loaded per round trip
+template <int kCombineBatch>
 __device__ __forceinline__ void merge_head_part(const DecodeParams& p, int b, const SplitList& sl,
                                                 int h, int d0) {
   // online merge: running max m, running weight sum l, running weighted sums v
@@ -1038,6 +1049,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     c.q_ready = 0;
     c.b_start = 0;
     c.off_start = 0;
+    c.L_start = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -1082,6 +1094,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
 
   // ---- plan (reads seq_lens: after the previous kernel has completed) -----
   griddep_wait();
+  if (tid == 0) MFA_TR(10, 0);
 #ifdef MFA_TRACE
   const int gt_call = blockIdx.x < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[blockIdx.x]) : -1;
   if (tid == 0) {
@@ -1091,34 +1104,44 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
   }
 #endif
   if (p.num_splits == 0) {
-    balanced_plan(p, c);  // ends with __syncthreads
-    if (tid == 0) {  // the next call's L2 warm-up hint
-      p.ws_hint[2 * blockIdx.x] = c.tiles > 0 ? c.b_start : -1;
-      p.ws_hint[2 * blockIdx.x + 1] = c.off_start;
-    }
+    balanced_plan(p, c);  // its plan words are fenced by their writers
   } else if (tid == 0) {
     c.tiles = static_cast<int>(blockIdx.x) < p.batch * p.num_splits ? -1 : 0;
     c.t0 = 0;
     c.ntot = 0;
-    fixed_plan_hint(p.seq_lens, p.cap_tokens, p.num_splits, p.ws_hint, c.tiles != 0);
   }
-  // This CTA owns the partial slots it may fill (balanced plan: 2c and 2c + 1;
-  // fixed split: units c, c + grid, ...): their flags start the call at zero.
-  if (p.num_splits == 0) {
-    if (tid < 2) p.ws_flag[2 * blockIdx.x + tid] = 0u;
-  } else {
-    const long long units = static_cast<long long>(p.batch) * p.num_splits;
-    for (long long u = blockIdx.x + static_cast<long long>(tid) * p.grid; u < units;
-         u += static_cast<long long>(kThreads) * p.grid)
-      p.ws_flag[u] = 0u;
-  }
-  // The plan words and cleared flags are in place before the combine kernel
-  // may start: it starts once every CTA of this grid has passed this trigger.
-  __threadfence();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_launch_dependents();
+  if (tid == 0) MFA_TR(10, 1);
+
+  // Set-up off the loaders' path, by the MMA warp (whose first products wait
+  // for q and the first K tile anyway): this CTA's partial slots (balanced
+  // plan: 2c and 2c + 1; fixed split: units c, c + grid, ...) start the call
+  // with cleared flags, the next call's L2 warm-up hint is written, and then
+  // the combine kernel may start: it starts once every CTA of this grid has
+  // passed the trigger (one thread's suffices for its CTA), so it never sees
+  // a flag of an earlier call or a plan word not yet written (those were
+  // fenced by their writers before the barrier above).
+  if (warp == 1) {
+    if (p.num_splits == 0) {
+      if (lane < 2) p.ws_flag[2 * blockIdx.x + lane] = 0u;
+      if (lane == 0) {
+        p.ws_hint[2 * blockIdx.x] = c.tiles > 0 ? c.b_start : -1;
+        p.ws_hint[2 * blockIdx.x + 1] = c.off_start;
+      }
+    } else {
+      const long long units = static_cast<long long>(p.batch) * p.num_splits;
+      for (long long u = blockIdx.x + static_cast<long long>(lane) * p.grid; u < units;
+           u += 32LL * p.grid)
+        p.ws_flag[u] = 0u;
+      if (lane == 0)
+        fixed_plan_hint(p.seq_lens, p.cap_tokens, p.num_splits, p.ws_hint, c.tiles != 0);
+    }
+    __threadfence();
+    __syncwarp();
+    griddep_launch_dependents();
+  }
 
   volatile int* abort_flag = &c.abort_flag;
   const uint32_t tmem = c.tmem_base;
@@ -1129,7 +1152,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     // ======================= K/V producer ===================================
     const uint64_t policy = l2_policy_evict_first();
     TileStream ks;
-    ks.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+    ks.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
     uint32_t item = 0;
 #ifdef MFA_TRACE
     int ntr[2] = {0, 0};
@@ -1224,6 +1247,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
             }
           }
           __syncwarp();
+          if (lane == 0) MFA_TR(13, item);
           ++item;
         }
         if (!ok) break;
@@ -1258,7 +1282,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     const uint32_t ring_base = smem_u32(sRing);
     const uint32_t p_base = smem_u32(sP);
     TileStream qs;
-    qs.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+    qs.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
     uint32_t nq = 0;
     bool ok = true;
     // Ring items, in the producer's order K0 | K1 V0 | K2 V1 | ... | V(T-1),
@@ -1416,6 +1440,14 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
           }
         }
       }
+#ifdef MFA_TRACE
+      if (g == 0 && have_cur) {  // first tile: when K(0), then q, is in place
+        wait_items(k_item(0));
+        if (lane == 0) MFA_TR(12, 2);
+        mbar_wait_warp(qbar, qpar, abort_flag);
+        if (lane == 0) MFA_TR(12, 1);
+      }
+#endif
       if (ok && need_qk) {
         ok = (!cur.seg_first || mbar_wait_warp(qbar, qpar, abort_flag)) &&
              (g < 2 || mbar_wait_warp(&c.s_empty[g & 1], par((g >> 1) - 1), abort_flag)) &&
@@ -1455,8 +1487,8 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     // is on its way, since k - 1's last PV is issued after k's first QK.
     const uint64_t policy = l2_policy_evict_last();
     TileStream qs, ahead;
-    qs.init(p, c.b_start, c.off_start, c.tiles, c.t0);
-    ahead.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+    qs.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
+    ahead.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
     TileInfo t, ta, last;
     bool more_ahead = ahead.next(ta);  // stays one segment ahead of qs
     bool have_last = false, ok = true;
@@ -1478,6 +1510,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
             for (int r = 0; r < 4; ++r)
               tma_load_3d(sQ + b * kQBytes + r * 8192, &tm_q, &c.q_full[b], r * 64, 0, t.b, policy);
           }
+          MFA_TR(12, 0);
         }
         // pull the next segment's q rows into L2 while this segment runs
         while (more_ahead && (ta.b == t.b || !ta.seg_first)) more_ahead = ahead.next(ta);
@@ -1520,7 +1553,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
       // through a four-entry ring (this warp runs at most two segments ahead
       // of them: q of the next segment waits for the current one's last QK).
       TileStream cs;
-      cs.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+      cs.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
       TileInfo t;
       uint32_t nq = 0;
       while (cs.next(t)) {
@@ -1546,7 +1579,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
       // After the softmax warps have written a segment's output or partial,
       // makes it visible device-wide and tells the combine kernel.
       TileStream ns;
-      ns.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+      ns.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
       TileInfo t;
       unsigned k = 0;
       while (ns.next(t)) {
@@ -1569,7 +1602,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     const int hl = lane & (kWGHeads - 1);
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
     TileStream ts;
-    ts.init(p, c.b_start, c.off_start, c.tiles, c.t0);
+    ts.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
     if (kFp8) {
       // the first segment's q conversion, with warp 3 (which publishes it)
       TileStream first = ts;
@@ -1909,7 +1942,14 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
 // attention kernel itself. One CTA waits for the attention grid to complete at
 // its end, so a call is over when this kernel is.
 // ===========================================================================
-__global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams p) {
+// kMinBlocks blocks per SM: 2 (128 registers, four partials per round trip)
+// or, for batches whose blocks would not all fit at two per SM, 4 (64
+// registers, two partials per round trip), so that a block waiting for a late
+// sequence does not keep a block of a finished one from starting.
+// (Measured: E4M3 batch 128, 71.3 -> 70.5 us with 4; bf16 batch 64, whose 256
+// blocks fit at 2 per SM, 54.3 -> 55.9 us with 4.)
+template <int kMinBlocks>
+__global__ void __launch_bounds__(kDim, kMinBlocks) mfa_combine_kernel(const DecodeParams p) {
 #ifdef MFA_TRACE
   const unsigned long long gt_start = global_timer_ns();
   const int cta_lin = blockIdx.x * gridDim.y + blockIdx.y;
@@ -1971,7 +2011,7 @@ __global__ void __launch_bounds__(kDim, 2) mfa_combine_kernel(const DecodeParams
         }
       }
       __syncthreads();
-      if (s_ok && dims_ok) merge_head_part(p, b, sl, h, d0);
+      if (s_ok && dims_ok) merge_head_part<kMinBlocks == 4 ? 2 : 4>(p, b, sl, h, d0);
     }
   }
   // One block waits for the attention grid to complete, so this grid never
@@ -2024,9 +2064,17 @@ static cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk
                     SmemLayout<kFp8>::kBytes, stream, tq, tk, tv, p);
 }
 
+// The combine variant for this batch (blocks per SM, above).
+static bool combine_wide(const DecodeParams& p) {
+  return static_cast<long long>(p.batch) * (kHeads / kCombineHeads) > 2LL * p.grid;
+}
+
 // The combine kernel alone, without programmatic launch (failure self-test).
 cudaError_t launch_combine_only(const DecodeParams& p, cudaStream_t stream) {
-  mfa_combine_kernel<<<dim3(p.batch, kHeads / kCombineHeads), dim3(kDim), 0, stream>>>(p);
+  if (combine_wide(p))
+    mfa_combine_kernel<4><<<dim3(p.batch, kHeads / kCombineHeads), dim3(kDim), 0, stream>>>(p);
+  else
+    mfa_combine_kernel<2><<<dim3(p.batch, kHeads / kCombineHeads), dim3(kDim), 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -2040,8 +2088,10 @@ cudaError_t launch_decode(bool paged, bool fp8, const CUtensorMap& tq, const CUt
     err = paged ? launch_attention<true, false>(tq, tk, tv, p, stream)
                 : launch_attention<false, false>(tq, tk, tv, p, stream);
   if (err != cudaSuccess) return err;
-  return launch_pdl(mfa_combine_kernel, dim3(p.batch, kHeads / kCombineHeads), dim3(kDim), 0,
-                    stream, p);
+  return combine_wide(p) ? launch_pdl(mfa_combine_kernel<4>, dim3(p.batch, kHeads / kCombineHeads),
+                                      dim3(kDim), 0, stream, p)
+                         : launch_pdl(mfa_combine_kernel<2>, dim3(p.batch, kHeads / kCombineHeads),
+                                      dim3(kDim), 0, stream, p);
 }
 
 }  // namespace mfa
