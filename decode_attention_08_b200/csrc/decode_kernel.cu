@@ -1092,8 +1092,10 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     }
   }
 
-  // ---- plan (reads seq_lens: after the previous kernel has completed) -----
-  griddep_wait();
+  // ---- plan (reads seq_lens: after the previous kernel has completed, or at
+  // once after the query projection, which launched this grid only after
+  // every kernel before it had completed) ----------------------------------
+  if (!p.q_after_proj) griddep_wait();
   if (tid == 0) MFA_TR(10, 0);
 #ifdef MFA_TRACE
   const int gt_call = blockIdx.x < kGtCtas ? *reinterpret_cast<volatile int*>(&g_mfa_cnt[blockIdx.x]) : -1;
@@ -1486,6 +1488,7 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     // converts there), one segment behind: segment k - 1 after q of segment k
     // is on its way, since k - 1's last PV is issued after k's first QK.
     const uint64_t policy = l2_policy_evict_last();
+    if (p.q_after_proj) griddep_wait();  // q is the projection grid's output
     TileStream qs, ahead;
     qs.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);
     ahead.init(p, c.b_start, c.off_start, c.tiles, c.t0, c.L_start);

@@ -342,7 +342,7 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
                 const mfa_tensor* page_table, const mfa_tensor* seq_lens, mfa_tensor* out,
                 float softmax_scale, int kv_dtype, float k_scale, float v_scale, int num_splits,
                 mfa_tensor* lse_out, void* workspace, size_t workspace_bytes, mfa_stream_t stream,
-                bool validate_only, bool gqa = false) {
+                bool validate_only, bool gqa = false, bool q_after_proj = false) {
   // ---- shapes and dtypes ----
   // grouped-query mode: q and out [B, 64, 128], caches [*, tokens, 2, 128] bf16,
   // viewed as [*, tokens, 256]
@@ -487,6 +487,7 @@ int decode_impl(const mfa_tensor* q, const mfa_tensor* k_cache, const mfa_tensor
   p.ws_flag = reinterpret_cast<unsigned*>(ws + wl.flag_off);
   p.wait_ns = kDecodeWaitNs;
   p.gqa = gqa ? 1 : 0;
+  p.q_after_proj = q_after_proj ? 1 : 0;
   const cudaError_t err =
       launch_decode(paged, fp8, tq, tk, tv, p, reinterpret_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? MFA_OK : cuda_fail(err);
@@ -685,12 +686,13 @@ int mfa_qproj_decode_attention(const mfa_tensor* x, const mfa_tensor* w_qa,
   if (!workspace || workspace_bytes < split + dbytes) return MFA_ERR_WORKSPACE;
   rc = qproj_impl(x, w_qa, w_qb, q_out, workspace, qbytes, stream, false);
   if (rc != MFA_OK) return rc;
-  // launched with programmatic dependent launch: its CTAs set up (barriers,
-  // TMEM, L2 warm-up of their first tiles) as the projection's CTAs finish,
-  // and read q only after the projection has completed
+  // launched with programmatic dependent launch as the projection's CTAs
+  // finish: the projection let it launch only after its own dependency wait,
+  // so the attention plans and streams K/V at once and waits for the
+  // projection grid only before it reads q
   return decode_impl(&q3, k_cache, v_cache, page_table, seq_lens, out, softmax_scale, kv_dtype,
                      k_scale, v_scale, num_splits, lse_out, static_cast<uint8_t*>(workspace) + split,
-                     workspace_bytes - split, stream, false);
+                     workspace_bytes - split, stream, false, false, true);
 }
 
 int mfa_query_proj(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,

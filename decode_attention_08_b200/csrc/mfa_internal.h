@@ -66,6 +66,11 @@ struct DecodeParams {
   // grouped-query mode (bf16 cache): q [B, 64, 128], key/value token rows
   // [2 groups][128], heads 0-31 in group 0 and 32-63 in group 1, out [B, 64, 128]
   int gqa;
+  // 1: the kernel launched just before this one on the stream is the query
+  // projection, which writes only q and lets this grid launch only after its
+  // own dependency wait. Every other input and the workspace are then ready at
+  // launch; only the q loader waits for the projection grid.
+  int q_after_proj;
 };
 
 struct QprojParams {

@@ -150,11 +150,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int stage_bytes = kABytes + n_cols * 128;
   GemmCtrl& c = *reinterpret_cast<GemmCtrl*>(smem + stages * stage_bytes);
 
-  // a kernel launched after this one with programmatic dependent launch (the
-  // decode attention after the up-projection, the key/value merge after the
-  // append projection) may set up as this grid's CTAs finish; it reads this
-  // grid's results only after it has completed
-  griddep_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m_tile = blockIdx.x;
   const int split = blockIdx.y;
@@ -183,6 +178,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // the previous kernel's tail; nothing in global memory is touched before it
   // has completed
   griddep_wait();
+  // A kernel launched after this one with programmatic dependent launch (the
+  // decode attention after the up-projection, the key/value merge after the
+  // append projection) may set up as this grid's CTAs finish; it reads this
+  // grid's results only after it has completed. The trigger follows the
+  // dependency wait, so that kernel starts only once every kernel before this
+  // one has completed (the projection -> attention call relies on it).
+  griddep_launch_dependents();
   const uint32_t tmem = c.tmem_base;
   volatile int* abort_flag = &c.abort_flag;
 
@@ -341,12 +343,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const int stages = fused_stages(stage_bytes);
   FusedCtrl& c = *reinterpret_cast<FusedCtrl*>(smem + stages * stage_bytes);
 
-  // A kernel launched after this one with programmatic dependent launch (the
-  // decode attention of mfa_qproj_decode_attention) may start its set-up as
-  // this grid's CTAs finish; it reads q only after this grid has completed.
-  // (It cannot take an SM before every CTA here has started: the trigger
-  // counts only once all of them have executed it.)
-  griddep_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool has1 = static_cast<int>(blockIdx.x) < p.m1_tiles * p.splits;
   const int tile1 = blockIdx.x % p.m1_tiles;
@@ -377,6 +373,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   // the previous kernel's tail; nothing in global memory is touched before it
   // has completed
   griddep_wait();
+  // A kernel launched after this one with programmatic dependent launch (the
+  // decode attention of mfa_qproj_decode_attention) may start as this grid's
+  // CTAs finish. The trigger follows the dependency wait: once it fires in
+  // every CTA, every kernel before this one has completed, so that attention
+  // kernel reads the lengths, the caches and its workspace at once and waits
+  // for this grid only before it reads q.
+  griddep_launch_dependents();
   const uint32_t tmem = c.tmem_base;
   volatile int* abort_flag = &c.abort_flag;
 
