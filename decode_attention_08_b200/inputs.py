@@ -305,7 +305,10 @@ WORKLOADS = {
     2: dict(name="mfa_decode_b64_l4096_bf16", batch=64, seq_len=4096),
     3: dict(name="mfa_paged_decode_b256_l1024-8192_p64_bf16", batch=256, seq_len=(1024, 8192),
             page_size=64),
-    4: dict(name="mfa_decode_b128_l4096_e4m3", batch=128, seq_len=4096, kv_dtype="e4m3"),
+    # uniform lengths, batch below the SM count: one CTA per sequence (no
+    # partials to merge) is the caller's split here
+    4: dict(name="mfa_decode_b128_l4096_e4m3", batch=128, seq_len=4096, kv_dtype="e4m3",
+            num_splits=1),
     5: dict(name="mfa_qproj_then_decode_b8_l65536_split16_bf16", batch=8, seq_len=65536,
             num_splits=16, qproj=True),
 }

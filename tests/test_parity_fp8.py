@@ -81,9 +81,13 @@ def test_fp8_fixed_splits():
 
 
 def test_workload4_fp8_all_outputs():
+    """Workload 4 at full size, in both launch configurations the benchmark
+    times: the balanced plan and one CTA per sequence (num_splits = 1)."""
     dec, _ = gen.make_workload(4)
-    got = run_decode(dec)
-    assert np.all(np.isfinite(got))
     ref, _ = oracle_decode(dec)
-    err = assert_close(got, ref, decode_atol(dec, ref, torch.float32, base=FP8_TOL), "wl4")
-    print(f"workload 4: max |err| {err:.2e} over {got.size} outputs")
+    tol = decode_atol(dec, ref, torch.float32, base=FP8_TOL)
+    for splits in (0, dec.meta["num_splits"]):
+        got = run_decode(dec, num_splits=splits)
+        assert np.all(np.isfinite(got))
+        err = assert_close(got, ref, tol, f"wl4 splits={splits}")
+        print(f"workload 4 (num_splits={splits}): max |err| {err:.2e} over {got.size} outputs")
