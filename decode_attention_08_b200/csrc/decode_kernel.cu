@@ -15,10 +15,13 @@
 // The probabilities enter the PV product as an exact-sum pair hi + lo (bf16
 // pair, or E4M3 pair with an FP8 cache) in one N = 128 product per step.
 //
-// CTA = 12 warps, one CTA per SM (persistent):
-//   warp 0       TMA producer for the K/V ring (4 slots x 32 KB)
+// CTA = 12 warps (bf16 cache; 20 with an FP8 cache, whose softmax runs in four
+// warpgroups of 16 heads), one CTA per SM (persistent):
+//   warp 0       TMA producer for the K/V ring (32 KB slots: 5 bf16, 4 FP8)
 //   warp 1       TMEM allocator + tcgen05.mma issuer (the whole warp runs the
-//                issue loop; elect.sync picks the issuing lane)
+//                issue loop; elect.sync picks the issuing lane); after the plan
+//                it also clears the CTA's partial flags and lets the combine
+//                kernel launch
 //   warp 2       TMA producer for q (one 32 KB load per sequence segment);
 //                with an FP8 cache also the segment publisher
 //   warp 3       bf16 cache: segment publisher; FP8 cache: q converter (q to
