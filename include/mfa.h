@@ -215,8 +215,9 @@ int mfa_query_proj(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor
  *   q_out = (x * W_qa) * W_qb            as mfa_query_proj_ex, q_out [B, 64 * 256]
  *   out   = attention(q_out viewed as [B, 64, 256], caches)   as mfa_decode_attention_ex
  * The projection writes q straight in the layout the attention reads, and the
- * attention kernel is launched with programmatic dependent launch: its CTAs set
- * up (barriers, TMEM, an L2 warm-up of their first key/value tiles) on the SMs
+ * attention kernel is launched with programmatic dependent launch: the
+ * projection lets it launch only after every earlier kernel on the stream has
+ * completed, so its CTAs plan and start streaming key/value tiles on the SMs
  * the projection's CTAs leave, and read q once the projection has completed.
  * workspace: mfa_qproj_decode_workspace_size(B, Dm, R, num_splits) bytes,
  * 256-byte aligned: the projection's workspace (its first 4 KB zero before the
@@ -239,8 +240,8 @@ size_t mfa_qproj_decode_workspace_size(int batch, int dm, int rank, int num_spli
  * mfa_query_proj_workspace_size(B, Dm, R) bytes, 256-byte aligned, that must be
  * zero-filled before its first use; every call returns its counters (the first
  * 4 KB) to zero, and the rest needs no initialisation. With B <= 8 both
- * products run in one persistent kernel that streams W_qb into L2 while the
- * latent is formed. */
+ * products run in one persistent kernel that fills its load ring with W_qb
+ * tiles while the latent is formed. */
 int mfa_query_proj_ex(const mfa_tensor* x, const mfa_tensor* w_qa, const mfa_tensor* w_qb,
                       mfa_tensor* q_out, void* workspace, size_t workspace_bytes,
                       mfa_stream_t stream);
