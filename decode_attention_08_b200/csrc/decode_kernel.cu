@@ -134,13 +134,16 @@ static_assert(offsetof(DecodeCtrl<false>, red) % 16 == 0 &&
 // Shared memory (1024-byte aligned base): q buffer(s) | ring | P | control.
 // bf16: one q buffer, five 32 KB ring slots (HBM-bound: every slot of bytes in
 // flight counts) and a 32 KB P tile (probabilities as a bf16 pair hi + lo, two
-// 16 KB column blocks). FP8: two q buffers, so the next segment's q is loaded
-// and converted a whole segment ahead, four ring slots and a 16 KB P tile (an
-// E4M3 pair, two 8 KB blocks).
-template <bool kFp8>
+// 16 KB column blocks). FP8: a 16 KB P tile (an E4M3 pair, two 8 KB blocks)
+// and either two q buffers, so the next segment's q is loaded and converted a
+// whole segment ahead, with four ring slots; or (kOneQ: every CTA has at most
+// one segment, as with a fixed split of no more units than CTAs) one q buffer
+// and five slots (measured, E4M3 batch 128 with one unit per sequence: 66.4 ->
+// 63.4 us; with several segments per CTA the second q buffer is worth more).
+template <bool kFp8, bool kOneQ = !kFp8>
 struct SmemLayout {
-  static constexpr int kQBufs = kFp8 ? 2 : 1;
-  static constexpr int kRing = kFp8 ? 4 : kSlots;
+  static constexpr int kQBufs = (kFp8 && !kOneQ) ? 2 : 1;
+  static constexpr int kRing = (kFp8 && !kOneQ) ? 4 : kSlots;
   static constexpr int kPSize = kFp8 ? kPBytes : 2 * kPBytes;
   static constexpr int kQ = 0;
   static constexpr int kRingOff = kQ + kQBufs * kQBytes;
@@ -148,9 +151,11 @@ struct SmemLayout {
   static constexpr int kCtrl = kP + kPSize;
   static constexpr int kBytes = kCtrl + static_cast<int>(sizeof(DecodeCtrl<kFp8>));
 };
-static_assert(SmemLayout<false>::kBytes <= 227 * 1024 && SmemLayout<true>::kBytes <= 227 * 1024,
+static_assert(SmemLayout<false>::kBytes <= 227 * 1024 && SmemLayout<true>::kBytes <= 227 * 1024 &&
+                  SmemLayout<true, true>::kBytes <= 227 * 1024,
               "shared memory budget");
-static_assert(SmemLayout<false>::kRing <= kSlots && SmemLayout<true>::kRing <= kSlots,
+static_assert(SmemLayout<false>::kRing <= kSlots && SmemLayout<true>::kRing <= kSlots &&
+                  SmemLayout<true, true>::kRing <= kSlots,
               "ring barriers");
 
 // bf16 P tile: the hi block and the lo block are 16 KB apart (the LBO of the
@@ -992,7 +997,7 @@ __device__ __noinline__ void segment_out(float* ws_o, void* out, int out_f32, in
 // ===========================================================================
 // the attention kernel
 // ===========================================================================
-template <bool kPaged, bool kFp8>
+template <bool kPaged, bool kFp8, bool kOneQ>
 __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     mfa_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -1000,8 +1005,10 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
   // 1024-byte alignment (the 128-byte swizzle atoms); checked below
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
-  using L = SmemLayout<kFp8>;
+  using L = SmemLayout<kFp8, kOneQ>;
   constexpr uint32_t kS = L::kRing;  // ring slots
+  // q buffer of the k-th segment (k & 1 with two buffers) and its phase parity
+  constexpr bool kTwoQ = L::kQBufs == 2;
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sRing = smem + L::kRingOff;
   uint8_t* sP = smem + L::kP;
@@ -1409,9 +1416,9 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     bool have_cur = qs.next(cur), pending_pv = false;
     while (ok && (have_cur || pending_pv)) {
       bool need_qk = have_cur, need_pv = pending_pv;
-      if (have_cur && cur.seg_first) qbuf = kFp8 ? (nq & 1u) : 0u;
+      if (have_cur && cur.seg_first) qbuf = kTwoQ ? (nq & 1u) : 0u;
       uint64_t* qbar = kFp8 ? &c.q_conv[qbuf] : &c.q_full[0];
-      const uint32_t qpar = kFp8 ? par(nq >> 1) : par(nq);
+      const uint32_t qpar = kTwoQ ? par(nq >> 1) : par(nq);
       if (kFp8 && need_qk && need_pv) {
         const uint64_t t0 = global_timer_ns();
         for (uint32_t spin = 1;; ++spin) {
@@ -1501,8 +1508,8 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
     uint32_t k = 0;
     while (ok && qs.next(t)) {
       if (t.seg_first) {
-        const uint32_t b = kFp8 ? (k & 1u) : 0u;
-        if (!(ok = mbar_wait_warp(&c.q_empty[b], (kFp8 ? par(k >> 1) : par(k)) ^ 1u, abort_flag))) break;
+        const uint32_t b = kTwoQ ? (k & 1u) : 0u;
+        if (!(ok = mbar_wait_warp(&c.q_empty[b], (kTwoQ ? par(k >> 1) : par(k)) ^ 1u, abort_flag))) break;
         if (lane == 0) {
           if (!kFp8 && p.gqa) {
             // boxes of 64 dims x 32 heads: group g's dims half r into q region
@@ -1564,8 +1571,8 @@ __global__ void __launch_bounds__(Geo<kFp8>::kThreads, 1)
       uint32_t nq = 0;
       while (cs.next(t)) {
         if (!t.seg_first) continue;
-        const uint32_t b = nq & 1u;  // q buffer of segment nq
-        const bool got = mbar_wait_warp(&c.q_full[b], par(nq >> 1), abort_flag);
+        const uint32_t b = kTwoQ ? (nq & 1u) : 0u;  // q buffer of segment nq
+        const bool got = mbar_wait_warp(&c.q_full[b], kTwoQ ? par(nq >> 1) : par(nq), abort_flag);
         // the first segment with the softmax warps (they call the same function)
         const float inv_s = nq == 0 ? q_to_e4m3_group(smem_u32(sQ), tid - 96, got, true, c.qmax)
                             : got   ? q_to_e4m3(smem_u32(sQ + b * kQBytes), lane)
@@ -2032,8 +2039,9 @@ __global__ void __launch_bounds__(kDim, kMinBlocks) mfa_combine_kernel(const Dec
 // host-side launch helper (called from mfa_api.cu)
 // ===========================================================================
 int decode_smem_bytes() {
-  return SmemLayout<false>::kBytes > SmemLayout<true>::kBytes ? SmemLayout<false>::kBytes
-                                                               : SmemLayout<true>::kBytes;
+  constexpr int a = SmemLayout<false>::kBytes, b = SmemLayout<true>::kBytes,
+                c = SmemLayout<true, true>::kBytes;
+  return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
 template <typename Kernel, typename... Args>
@@ -2052,7 +2060,7 @@ static cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <bool kPaged, bool kFp8>
+template <bool kPaged, bool kFp8, bool kOneQ>
 static cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk,
                                     const CUtensorMap& tv, const DecodeParams& p,
                                     cudaStream_t stream) {
@@ -2061,13 +2069,14 @@ static cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
     const cudaError_t err = cudaFuncSetAttribute(
-        mfa_decode_kernel<kPaged, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        SmemLayout<kFp8>::kBytes);
+        mfa_decode_kernel<kPaged, kFp8, kOneQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SmemLayout<kFp8, kOneQ>::kBytes);
     if (err != cudaSuccess) return err;
     configured_dev = dev;
   }
-  return launch_pdl(mfa_decode_kernel<kPaged, kFp8>, dim3(p.grid), dim3(Geo<kFp8>::kThreads),
-                    SmemLayout<kFp8>::kBytes, stream, tq, tk, tv, p);
+  return launch_pdl(mfa_decode_kernel<kPaged, kFp8, kOneQ>, dim3(p.grid),
+                    dim3(Geo<kFp8>::kThreads), SmemLayout<kFp8, kOneQ>::kBytes, stream, tq, tk,
+                    tv, p);
 }
 
 // The combine variant for this batch (blocks per SM, above).
@@ -2087,12 +2096,18 @@ cudaError_t launch_combine_only(const DecodeParams& p, cudaStream_t stream) {
 cudaError_t launch_decode(bool paged, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                           const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
   cudaError_t err;
-  if (fp8)
-    err = paged ? launch_attention<true, true>(tq, tk, tv, p, stream)
-                : launch_attention<false, true>(tq, tk, tv, p, stream);
+  // FP8 with at most one unit (so one segment) per CTA: one q buffer, a deeper ring
+  const bool one_q =
+      p.num_splits > 0 && static_cast<long long>(p.batch) * p.num_splits <= p.grid;
+  if (fp8 && one_q)
+    err = paged ? launch_attention<true, true, true>(tq, tk, tv, p, stream)
+                : launch_attention<false, true, true>(tq, tk, tv, p, stream);
+  else if (fp8)
+    err = paged ? launch_attention<true, true, false>(tq, tk, tv, p, stream)
+                : launch_attention<false, true, false>(tq, tk, tv, p, stream);
   else
-    err = paged ? launch_attention<true, false>(tq, tk, tv, p, stream)
-                : launch_attention<false, false>(tq, tk, tv, p, stream);
+    err = paged ? launch_attention<true, false, true>(tq, tk, tv, p, stream)
+                : launch_attention<false, false, true>(tq, tk, tv, p, stream);
   if (err != cudaSuccess) return err;
   return combine_wide(p) ? launch_pdl(mfa_combine_kernel<4>, dim3(p.batch, kHeads / kCombineHeads),
                                       dim3(kDim), 0, stream, p)
