@@ -50,8 +50,10 @@ def test_fp8_ragged_contiguous(out_dtype):
     assert err < FP8_TOL
 
 
-@pytest.mark.parametrize("page_size", [16, 64, 256])
-def test_fp8_paged_is_bit_exact_with_contiguous(page_size):
+@pytest.mark.parametrize("page_size,num_splits", [(16, 0), (64, 0), (256, 0), (64, 3)])
+def test_fp8_paged_is_bit_exact_with_contiguous(page_size, num_splits):
+    """Paged and contiguous caches give identical bits; num_splits = 3 (6 x 3 units,
+    fewer than the CTAs) runs the one-q-buffer, five-slot FP8 kernels."""
     lens = [1, 65, 200, 1000, 4097, 129]
     dec = gen.make_decode_inputs(503 + page_size, len(lens), lens, page_size=page_size,
                                  kv_dtype="e4m3")
@@ -65,8 +67,8 @@ def test_fp8_paged_is_bit_exact_with_contiguous(page_size):
         vc[b, :L] = dec.v[pages, t % page_size]
     cont = gen.DecodeInputs(q=dec.q, k=kc, v=vc, seq_lens=dec.seq_lens, kv_dtype="e4m3",
                             k_scale=dec.k_scale, v_scale=dec.v_scale)
-    got_p = run_decode(dec)
-    got_c = run_decode(cont)
+    got_p = run_decode(dec, num_splits=num_splits)
+    got_c = run_decode(cont, num_splits=num_splits)
     assert np.array_equal(got_p, got_c)
     ref, _ = oracle_decode(dec)
     assert_close(got_p, ref, decode_atol(dec, ref, torch.float32, base=FP8_TOL), "fp8 paged")
